@@ -1,0 +1,291 @@
+// The C-ABI entry points of libaal: argument checks, path choice, launches.
+#include <string.h>
+
+#include "aal_internal.h"
+
+namespace aal {
+
+static thread_local int t_policy = AAL_PATH_AUTO;
+static thread_local int t_last_path = 0;
+static thread_local long long t_launches = 0;
+
+void note_launch(int n) { t_launches += n; }
+void note_path(int path) { t_last_path = path; }
+
+static thread_local cudaEvent_t t_ev_before[8] = {};
+static thread_local cudaEvent_t t_ev_after[8] = {};
+
+// Records the one-shot timing events of ``kind`` around ``launch``.
+template <typename F>
+static aal_status timed(int kind, cudaStream_t s, F launch) {
+  cudaEvent_t b = t_ev_before[kind], a = t_ev_after[kind];
+  if (b && cudaEventRecord(b, s) != cudaSuccess) return AAL_ERR_CUDA;
+  aal_status st = launch();
+  if (a && st == AAL_OK && cudaEventRecord(a, s) != cudaSuccess) return AAL_ERR_CUDA;
+  if (st == AAL_OK) { t_ev_before[kind] = nullptr; t_ev_after[kind] = nullptr; }
+  return st;
+}
+
+static bool valid_law(int law, int q) {
+  if (q < 1 || q > (1 << 16)) return false;
+  if (law == AAL_LAW_Q) return true;
+  if (law == AAL_LAW_Q2XQ2) return q == 4;
+  return false;
+}
+
+static bool valid_mat(const aal_mat& m) {
+  if (m.dtype != AAL_BF16 && m.dtype != AAL_F32) return false;
+  if (m.rows < 0 || m.cols < 0 || m.ld < m.cols || m.ld < 0) return false;
+  if (m.rows > 0 && m.cols > 0 && m.ptr == nullptr) return false;
+  const size_t es = m.dtype == AAL_F32 ? 4 : 2;
+  if (m.ptr && ((uintptr_t)m.ptr % es) != 0) return false;
+  return true;
+}
+
+static bool valid_rule(const aal_row_type_rule& r, long long rows) {
+  if (r.kind == AAL_TYPES_POSITION) return r.seq_len > 0 && r.pos_offset >= 0;
+  if (r.kind == AAL_TYPES_EXPLICIT) return rows == 0 || r.types != nullptr;
+  return false;
+}
+
+static RowTypes make_types(const aal_row_type_rule& r, int q) {
+  RowTypes rt;
+  rt.kind = r.kind == AAL_TYPES_POSITION ? kTypesPosition : kTypesExplicit;
+  rt.q = q;
+  rt.seq_len = r.seq_len > 0 ? r.seq_len : 1;
+  rt.pos_offset = r.pos_offset;
+  rt.types = r.types;
+  rt.positions = nullptr;
+  return rt;
+}
+
+// Runs the tensor-core launcher when the policy allows it, else the general
+// one.  ``tc`` returns AAL_ERR_UNSUPPORTED without launching anything when it
+// cannot serve the shape.
+template <typename TC, typename GEN>
+static aal_status dispatch(int kind, cudaStream_t s, TC tc_launch, GEN gen_launch) {
+  auto tc = [&] { return timed(kind, s, tc_launch); };
+  auto gen = [&] { return timed(kind, s, gen_launch); };
+  if (t_policy != AAL_PATH_GENERAL) {
+    aal_status st = tc();
+    if (st == AAL_OK) { note_path(AAL_PATH_TENSOR); return AAL_OK; }
+    if (st != AAL_ERR_UNSUPPORTED || t_policy == AAL_PATH_TENSOR) return st;
+  }
+  aal_status st = gen();
+  if (st == AAL_OK) note_path(AAL_PATH_GENERAL);
+  return st;
+}
+
+}  // namespace aal
+
+using namespace aal;
+
+extern "C" {
+
+aal_status aal_project_fwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_mat X, aal_mat W,
+                           aal_mat Y, void* stream) {
+  if (!valid_law(law, q) || !valid_mat(X) || !valid_mat(W) || !valid_mat(Y))
+    return AAL_ERR_INVALID_ARG;
+  if (X.dtype != W.dtype || X.dtype != Y.dtype) return AAL_ERR_UNSUPPORTED;
+  if (W.rows != X.cols || Y.rows != X.rows || Y.cols != W.cols) return AAL_ERR_INVALID_ARG;
+  if (X.cols % q || W.cols % q) return AAL_ERR_INVALID_ARG;
+  if (!valid_rule(rule, X.rows)) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (X.rows == 0 || Y.cols == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  RowTypes rt = make_types(rule, q);
+  return dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, X.rows, X, W, Y, s); },
+                  [&] { return simt_project(law, q, rt, X, W, Y, s); });
+}
+
+aal_status aal_swiglu_fwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_mat X, aal_mat Wg,
+                          aal_mat Wu, aal_mat Wd, aal_mat H, aal_mat Y, void* stream) {
+  if (!valid_law(law, q) || !valid_mat(X) || !valid_mat(Wg) || !valid_mat(Wu) ||
+      !valid_mat(Wd) || !valid_mat(H) || !valid_mat(Y))
+    return AAL_ERR_INVALID_ARG;
+  const int dt = X.dtype;
+  if (Wg.dtype != dt || Wu.dtype != dt || Wd.dtype != dt || H.dtype != dt || Y.dtype != dt)
+    return AAL_ERR_UNSUPPORTED;
+  const long long M = X.rows, D = X.cols, F = Wg.cols;
+  if (Wg.rows != D || Wu.rows != D || Wu.cols != F || Wd.rows != F || Wd.cols != D ||
+      H.rows != M || H.cols != F || Y.rows != M || Y.cols != D)
+    return AAL_ERR_INVALID_ARG;
+  if (D % q || F % q) return AAL_ERR_INVALID_ARG;
+  if (!valid_rule(rule, M)) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (M == 0 || D == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  RowTypes rt = make_types(rule, q);
+  int path_gu = 0;
+  aal_status st = dispatch(AAL_KERNEL_GATE_UP, s, [&] { return tc_swiglu_gate_up(law, q, rt, M, X, Wg, Wu, H, s); },
+                           [&] { return simt_swiglu_gate_up(law, q, rt, X, Wg, Wu, H, s); });
+  if (st != AAL_OK) return st;
+  path_gu = t_last_path;
+  st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, H, Wd, Y, s); },
+                [&] { return simt_project(law, q, rt, H, Wd, Y, s); });
+  if (st == AAL_OK && path_gu != t_last_path) note_path(AAL_PATH_GENERAL);
+  return st;
+}
+
+aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_mat X, aal_mat W,
+                           aal_mat dY, aal_mat dX, aal_mat dW, int32_t accumulate_dW,
+                           void* stream) {
+  if (!valid_law(law, q) || !valid_mat(X) || !valid_mat(W) || !valid_mat(dY))
+    return AAL_ERR_INVALID_ARG;
+  const bool want_dx = dX.ptr != nullptr, want_dw = dW.ptr != nullptr;
+  if ((want_dx && !valid_mat(dX)) || (want_dw && !valid_mat(dW))) return AAL_ERR_INVALID_ARG;
+  const int dt = X.dtype;
+  if (W.dtype != dt || dY.dtype != dt || (want_dx && dX.dtype != dt) ||
+      (want_dw && dW.dtype != dt))
+    return AAL_ERR_UNSUPPORTED;
+  const long long M = X.rows, din = X.cols, dout = W.cols;
+  if (W.rows != din || dY.rows != M || dY.cols != dout) return AAL_ERR_INVALID_ARG;
+  if (want_dx && (dX.rows != M || dX.cols != din)) return AAL_ERR_INVALID_ARG;
+  if (want_dw && (dW.rows != din || dW.cols != dout)) return AAL_ERR_INVALID_ARG;
+  if (din % q || dout % q) return AAL_ERR_INVALID_ARG;
+  if (!valid_rule(rule, M)) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  cudaStream_t s = (cudaStream_t)stream;
+  RowTypes rt = make_types(rule, q);
+  int paths = 0;
+  if (want_dx && M > 0 && din > 0) {
+    aal_status st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dY, W, dX, s); },
+                             [&] { return simt_project_bwd_dx(law, q, rt, dY, W, dX, s); });
+    if (st != AAL_OK) return st;
+    paths |= 1 << t_last_path;
+  }
+  if (want_dw && din > 0 && dout > 0) {
+    aal_status st =
+        dispatch(AAL_KERNEL_BWD_DW, s, [&] { return tc_project_bwd_dw(law, q, rt, M, X, dY, dW, accumulate_dW, s); },
+                 [&] { return simt_project_bwd_dw(law, q, rt, X, dY, dW, accumulate_dW, s); });
+    if (st != AAL_OK) return st;
+    paths |= 1 << t_last_path;
+  }
+  if (paths) note_path((paths & (1 << AAL_PATH_GENERAL)) ? AAL_PATH_GENERAL : AAL_PATH_TENSOR);
+  return AAL_OK;
+}
+
+aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* positions, aal_mat x,
+                             aal_mat W, aal_mat y, void* stream) {
+  if (!valid_law(law, q) || !valid_mat(x) || !valid_mat(W) || !valid_mat(y))
+    return AAL_ERR_INVALID_ARG;
+  if (x.dtype != W.dtype || x.dtype != y.dtype) return AAL_ERR_UNSUPPORTED;
+  if (W.rows != x.cols || y.rows != x.rows || y.cols != W.cols) return AAL_ERR_INVALID_ARG;
+  if (x.cols % q || W.cols % q) return AAL_ERR_INVALID_ARG;
+  if (x.rows > 0 && positions == nullptr) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (x.rows == 0 || y.cols == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (t_policy != AAL_PATH_GENERAL) {
+    bool handled = false;
+    aal_status st = timed(AAL_KERNEL_DECODE, s, [&] {
+      return decode_matvec(law, q, positions, x, W, y, s, &handled);
+    });
+    if (handled) {
+      if (st == AAL_OK) note_path(AAL_PATH_DECODE);
+      return st;
+    }
+    if (t_policy == AAL_PATH_TENSOR) return AAL_ERR_UNSUPPORTED;
+  }
+  RowTypes rt;
+  rt.kind = kTypesPositions64;
+  rt.q = q;
+  rt.seq_len = 1;
+  rt.pos_offset = 0;
+  rt.types = nullptr;
+  rt.positions = positions;
+  aal_status st = simt_project(law, q, rt, x, W, y, s);
+  if (st == AAL_OK) note_path(AAL_PATH_GENERAL);
+  return st;
+}
+
+aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat W, aal_mat Z,
+                              void* stream) {
+  if (!valid_law(law, q) || !valid_mat(X) || !valid_mat(W) || !valid_mat(Z))
+    return AAL_ERR_INVALID_ARG;
+  if (X.dtype != W.dtype || X.dtype != Z.dtype) return AAL_ERR_UNSUPPORTED;
+  const long long n = X.rows;
+  if (X.cols != n || W.rows != n || W.cols != n || Z.rows != n || Z.cols != n)
+    return AAL_ERR_INVALID_ARG;
+  if (n % q) return AAL_ERR_INVALID_ARG;
+  if (n > 0 && (Z.ptr == X.ptr || Z.ptr == W.ptr)) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (n == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  return dispatch(AAL_KERNEL_SQUARE, s, [&] { return tc_square(law, q, X, W, Z, s); },
+                  [&] { return simt_square(law, q, X, W, Z, s); });
+}
+
+aal_status aal_block_table(int32_t law, int32_t q, uint8_t* S) {
+  if (!valid_law(law, q) || S == nullptr) return AAL_ERR_INVALID_ARG;
+  for (int i = 0; i < q; ++i)
+    for (int k = 0; k < q; ++k)
+      for (int a = 0; a < q; ++a)
+        S[((size_t)i * q + k) * q + a] = in_table(law, i, k, a) ? 1 : 0;
+  return AAL_OK;
+}
+
+int64_t aal_block_product_count(int32_t law, int32_t q, int32_t row_typed) {
+  if (!valid_law(law, q)) return -1;
+  int64_t n = 0;
+  const int rows = row_typed ? 1 : q;
+  for (int i = 0; i < rows; ++i)
+    for (int k = 0; k < q; ++k) {
+      int members[4];
+      n += table_members(law, q, i, k, members);
+    }
+  return n;
+}
+
+aal_status aal_get_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return AAL_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpyFromSymbol(&code, g_device_status, sizeof(int)) != cudaSuccess)
+    return AAL_ERR_CUDA;
+  if (code != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return AAL_ERR_CUDA;
+  }
+  if (code == kDevTimeout) return AAL_ERR_DEVICE_TIMEOUT;
+  if (code == kDevBounds) return AAL_ERR_DEVICE_BOUNDS;
+  return AAL_OK;
+}
+
+const char* aal_status_string(int32_t status) {
+  switch (status) {
+    case AAL_OK: return "ok";
+    case AAL_ERR_INVALID_ARG: return "invalid argument";
+    case AAL_ERR_UNSUPPORTED: return "unsupported by this build";
+    case AAL_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case AAL_ERR_CUDA: return "CUDA runtime error";
+    case AAL_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+    case AAL_ERR_DEVICE_BOUNDS: return "a kernel met an out-of-range row type or position";
+    default: return "unknown status";
+  }
+}
+
+aal_status aal_set_timing_events(int32_t kernel, void* before, void* after) {
+  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_DECODE) return AAL_ERR_INVALID_ARG;
+  t_ev_before[kernel] = (cudaEvent_t)before;
+  t_ev_after[kernel] = (cudaEvent_t)after;
+  return AAL_OK;
+}
+
+aal_status aal_set_path_policy(int32_t policy) {
+  if (policy < AAL_PATH_AUTO || policy > AAL_PATH_GENERAL) return AAL_ERR_INVALID_ARG;
+  t_policy = policy;
+  return AAL_OK;
+}
+
+int32_t aal_last_path(void) { return t_last_path; }
+
+int64_t aal_launch_count(int32_t reset) {
+  const long long n = t_launches;
+  if (reset) t_launches = 0;
+  return n;
+}
+
+int32_t aal_version(void) { return 100; }
+
+}  // extern "C"

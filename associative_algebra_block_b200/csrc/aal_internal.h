@@ -1,0 +1,109 @@
+// Internal declarations shared by the libaal translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "aal.h"
+
+namespace aal {
+
+// Device status word (one per device that loaded the library).  Kernels set it
+// with atomicCAS from 0 so the first error wins; aal_get_device_status reads
+// and clears it.  Defined here: the library is a single translation unit.
+enum DeviceCode : int { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
+__device__ int g_device_status = 0;
+
+__device__ __forceinline__ void flag_device_error(int code) {
+  atomicCAS(&g_device_status, 0, code);
+}
+
+// Where a row's type comes from.
+enum RowTypeKind : int { kTypesPosition = 0, kTypesExplicit = 1, kTypesPositions64 = 2 };
+
+struct RowTypes {
+  int kind;
+  int q;
+  long long seq_len;
+  long long pos_offset;
+  const int32_t* types;      // kind 1
+  const int64_t* positions;  // kind 2 (decode)
+};
+
+// Row type of row r; -1 (and the bounds flag) for an explicit type outside
+// [0, q) or a negative position.
+__device__ __forceinline__ int row_type(const RowTypes& rt, long long r) {
+  if (rt.kind == kTypesPosition) {
+    return (int)(((r % rt.seq_len) + rt.pos_offset) % rt.q);
+  }
+  if (rt.kind == kTypesExplicit) {
+    int t = rt.types[r];
+    if (t < 0 || t >= rt.q) { flag_device_error(kDevBounds); return -1; }
+    return t;
+  }
+  long long p = rt.positions[r];
+  if (p < 0) { flag_device_error(kDevBounds); return -1; }
+  return (int)(p % rt.q);
+}
+
+// Membership a in S(t, k) of the multiplication table.
+//  Q_q:      S(t, t) = {t}, S(t, k) = {t, k}
+//  Q2 x Q2:  groups are pairs g = 2*g1 + g2 and membership factorises.
+__host__ __device__ __forceinline__ bool in_table(int law, int t, int k, int a) {
+  if (law == AAL_LAW_Q) return a == t || a == k;
+  const int t1 = t >> 1, t2 = t & 1, k1 = k >> 1, k2 = k & 1, a1 = a >> 1, a2 = a & 1;
+  return (a1 == t1 || a1 == k1) && (a2 == t2 || a2 == k2);
+}
+
+// The members of S(t, k) in ascending order; returns their count (1, 2 or 4).
+__host__ __device__ __forceinline__ int table_members(int law, int q, int t, int k, int* a) {
+  if (law == AAL_LAW_Q) {
+    if (t == k) { a[0] = t; return 1; }
+    a[0] = t < k ? t : k;
+    a[1] = t < k ? k : t;
+    return 2;
+  }
+  int n = 0;
+  for (int g = 0; g < q; ++g)
+    if (in_table(law, t, k, g)) a[n++] = g;
+  return n;
+}
+
+// Per-thread launch accounting and path bookkeeping (api.cu).
+void note_launch(int n = 1);
+void note_path(int path);
+
+// ---------------------------------------------------------------- general path
+aal_status simt_project(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& W,
+                        const aal_mat& Y, cudaStream_t s);
+aal_status simt_swiglu_gate_up(int law, int q, const RowTypes& rt, const aal_mat& X,
+                               const aal_mat& Wg, const aal_mat& Wu, const aal_mat& H, cudaStream_t s);
+aal_status simt_project_bwd_dx(int law, int q, const RowTypes& rt, const aal_mat& dY,
+                               const aal_mat& W, const aal_mat& dX, cudaStream_t s);
+aal_status simt_project_bwd_dw(int law, int q, const RowTypes& rt, const aal_mat& X,
+                               const aal_mat& dY, const aal_mat& dW, int accumulate, cudaStream_t s);
+aal_status simt_square(int law, int q, const aal_mat& X, const aal_mat& W, const aal_mat& Z,
+                       cudaStream_t s);
+
+// ----------------------------------------------------------------- decode path
+aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
+                         const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled);
+
+// ------------------------------------------------------------ tensor-core path
+// Each returns AAL_ERR_UNSUPPORTED (launching nothing) when the shape is not
+// one the tensor-core kernels serve.
+aal_status tc_project(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                      const aal_mat& W, const aal_mat& Y, cudaStream_t s);
+aal_status tc_swiglu_gate_up(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                             const aal_mat& Wg, const aal_mat& Wu, const aal_mat& H, cudaStream_t s);
+aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
+                             const aal_mat& W, const aal_mat& dX, cudaStream_t s);
+aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                             const aal_mat& dY, const aal_mat& dW, int accumulate, cudaStream_t s);
+aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const aal_mat& Z,
+                     cudaStream_t s);
+
+inline aal_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AAL_OK : AAL_ERR_CUDA; }
+
+}  // namespace aal

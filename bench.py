@@ -1,0 +1,527 @@
+#!/usr/bin/env python3
+"""Benchmark of the associative-algebra block projections (libaal) on B200.
+
+Default workload: the Q2 (x) Q2 SwiGLU FFN of the 110M pilot (d = 768,
+ffn = 1536, 8 packed sequences of 1536 tokens = 12288 tokens, bf16) — one
+step is the full algebraic SwiGLU forward over those tokens plus the decode
+matrix-vector products of the three FFN projections at batch 1, 8 and 64.
+Metric: executed bf16 TFLOP/s (2 x the block MACs the table requires), with
+the fraction of the measured tensor peak and the speedup over a same-shape
+dense torch.matmul on the same GPU.
+
+Contract: ``python bench.py --gpus N --steps K --warmup W`` prints ONE JSON
+line on rank 0.  Under torchrun every rank runs the same per-GPU workload on
+its own tokens (token sharding, weights replicated, no collective on the
+data path: weak scaling); the time is the max over ranks.
+``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import associative_algebra_block_b200 as aal  # noqa: E402
+from associative_algebra_block_b200 import inputs  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# Workloads
+# ---------------------------------------------------------------------------
+
+def _exec_flops_proj(law, q, M, din, dout):
+    per_row = aal.aal_block_product_count(law, q, True)
+    return 2 * M * (din // q) * (dout // q) * per_row
+
+
+class SwigluDecode:
+    """Algebraic SwiGLU forward over M packed tokens + decode matvecs."""
+
+    def __init__(self, name, law, q, M, D, F, seq_len, w_sigma_rule="din", decode_batches=(1, 8, 64)):
+        self.name, self.law, self.q, self.M, self.D, self.F = name, law, q, M, D, F
+        self.seq_len, self.w_sigma_rule, self.decode_batches = seq_len, w_sigma_rule, decode_batches
+        f_gu = _exec_flops_proj(law, q, M, D, F)
+        f_d = _exec_flops_proj(law, q, M, F, D)
+        self.gate_up_flops = 2 * f_gu
+        self.fwd_flops = 2 * f_gu + f_d
+        self.dec_flops = sum(2 * _exec_flops_proj(law, q, B, D, F) + _exec_flops_proj(law, q, B, F, D)
+                             for B in decode_batches)
+        self.exec_flops = self.fwd_flops + self.dec_flops
+        self.dense_flops = 2 * M * D * F * 3 + sum(2 * B * D * F * 3 for B in decode_batches)
+        self.dominant = aal.AAL_KERNEL_GATE_UP
+        self.dominant_flops = self.gate_up_flops
+        self.dominant_name = "gate_up (fused gate/up projections + SiLU*mul)"
+
+    def config(self):
+        return {"workload": f"{self.name}: {self.law} q={self.q} SwiGLU FFN fwd d={self.D} "
+                            f"ffn={self.F} M={self.M} ({self.M // self.seq_len}x{self.seq_len} tokens) "
+                            f"+ decode matvec B={'/'.join(map(str, self.decode_batches))}",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F,
+                "seq_len": self.seq_len, "decode_batches": list(self.decode_batches)}
+
+    def bytes_per_set(self):
+        e = 2
+        w = 3 * self.D * self.F * e
+        act = self.M * (2 * self.D + self.F) * e
+        return w + act
+
+    def setup(self, nsets, seed):
+        ins = inputs.swiglu_inputs(self.D, self.F, self.M, seed=seed, dtype="bf16",
+                                   w_sigma_rule=self.w_sigma_rule, want_f64=False)
+        self.host_X = ins["X"].t
+        self.sets = []
+        for i in range(nsets):
+            s = {k: ins[k].t.cuda() for k in ("X", "Wg", "Wu", "Wd")}
+            s["H"] = torch.empty(self.M, self.F, dtype=torch.bfloat16, device="cuda")
+            s["Y"] = torch.empty(self.M, self.D, dtype=torch.bfloat16, device="cuda")
+            s["dec"] = []
+            st = inputs.Stream(seed + 100 + i)
+            for B in self.decode_batches:
+                x = st.normal(B, self.D, 1.0, "bf16", want_f64=False).t.cuda()
+                h = st.normal(B, self.F, 1.0, "bf16", want_f64=False).t.cuda()
+                pos = torch.from_numpy(st.positions(B, self.seq_len)).cuda()
+                s["dec"].append(dict(x=x, h=h, pos=pos,
+                                     g=torch.empty(B, self.F, dtype=torch.bfloat16, device="cuda"),
+                                     u=torch.empty(B, self.F, dtype=torch.bfloat16, device="cuda"),
+                                     y=torch.empty(B, self.D, dtype=torch.bfloat16, device="cuda")))
+            self.sets.append(s)
+        self.rule = aal.row_rule(seq_len=self.seq_len)
+        # pinned host copies for the end-to-end leg
+        self.pin = dict(X=self.host_X.pin_memory(),
+                        Y=torch.empty(self.M, self.D, dtype=torch.bfloat16).pin_memory(),
+                        dec=[dict(x=d["x"].cpu().pin_memory(), pos=d["pos"].cpu().pin_memory(),
+                                  h=d["h"].cpu().pin_memory(),
+                                  g=torch.empty_like(d["g"], device="cpu").pin_memory(),
+                                  u=torch.empty_like(d["u"], device="cpu").pin_memory(),
+                                  y=torch.empty_like(d["y"], device="cpu").pin_memory())
+                             for d in self.sets[0]["dec"]])
+
+    def step(self, i, ev=None):
+        s = self.sets[i % len(self.sets)]
+        if ev is not None:
+            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
+        aal.aal_swiglu_fwd(self.law, self.q, self.rule, s["X"], s["Wg"], s["Wu"], s["Wd"], s["H"], s["Y"])
+        for d in s["dec"]:
+            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["x"], s["Wg"], d["g"])
+            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["x"], s["Wu"], d["u"])
+            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["h"], s["Wd"], d["y"])
+
+    def dense_step(self, i):
+        s = self.sets[i % len(self.sets)]
+        torch.matmul(s["X"], s["Wg"], out=s["H"])
+        torch.matmul(s["X"], s["Wu"], out=s["H"])
+        torch.matmul(s["H"], s["Wd"], out=s["Y"])
+        for d in s["dec"]:
+            torch.matmul(d["x"], s["Wg"], out=d["g"])
+            torch.matmul(d["x"], s["Wu"], out=d["u"])
+            torch.matmul(d["h"], s["Wd"], out=d["y"])
+
+    def e2e_step(self, i):
+        """Host -> device inputs, the calls, device -> host results."""
+        s = self.sets[i % len(self.sets)]
+        p = self.pin
+        s["X"].copy_(p["X"], non_blocking=True)
+        for d, hd in zip(s["dec"], p["dec"]):
+            d["x"].copy_(hd["x"], non_blocking=True)
+            d["h"].copy_(hd["h"], non_blocking=True)
+            d["pos"].copy_(hd["pos"], non_blocking=True)
+        self.step(i)
+        p["Y"].copy_(s["Y"], non_blocking=True)
+        for d, hd in zip(s["dec"], p["dec"]):
+            hd["g"].copy_(d["g"], non_blocking=True)
+            hd["u"].copy_(d["u"], non_blocking=True)
+            hd["y"].copy_(d["y"], non_blocking=True)
+
+    def e2e_bytes(self):
+        h2d = self.M * self.D * 2 + sum(B * (self.D + self.F) * 2 + B * 8 for B in self.decode_batches)
+        d2h = self.M * self.D * 2 + sum(B * (2 * self.F + self.D) * 2 for B in self.decode_batches)
+        return h2d, d2h
+
+    # ---- oracle sample for the CPU baseline / reference arm
+    def oracle_sample(self, rows):
+        import oracle
+        s = inputs.swiglu_inputs(self.D, self.F, self.M, seed=0, dtype="bf16",
+                                 w_sigma_rule=self.w_sigma_rule)
+        types = oracle.row_types(self.law, self.q, inputs.packed_positions(self.M, self.seq_len))
+        st = inputs.Stream(100)
+        dec = []
+        for B in self.decode_batches:
+            dec.append((st.normal(B, self.D, 1.0, "bf16").f64, st.normal(B, self.F, 1.0, "bf16").f64,
+                        st.positions(B, self.seq_len)))
+        rows = min(rows, self.M)
+        sel = np.arange(rows) * (self.M // rows)
+        flops = (self.fwd_flops * rows) // self.M + self.dec_flops
+
+        def run():
+            oracle.swiglu_rows(self.law, self.q, types, s["X"].f64, s["Wg"].f64, s["Wu"].f64,
+                               s["Wd"].f64, sel)
+            for x, h, pos in dec:
+                oracle.decode(self.law, self.q, pos, x, s["Wg"].f64)
+                oracle.decode(self.law, self.q, pos, x, s["Wu"].f64)
+                oracle.decode(self.law, self.q, pos, h, s["Wd"].f64)
+
+        desc = (f"oracle SwiGLU forward on {rows} of {self.M} rows (evenly strided, all row types) "
+                f"+ the full decode matvecs B={'/'.join(map(str, self.decode_batches))}")
+        return flops, run, desc
+
+
+class ProjFwdBwd:
+    """Q_16 narrow FFN (expert-shaped): forward and backward of the gate/up
+    shaped and down shaped projections."""
+
+    def __init__(self, name, law, q, M, D, F, seq_len):
+        self.name, self.law, self.q, self.M, self.D, self.F, self.seq_len = name, law, q, M, D, F, seq_len
+        f1 = _exec_flops_proj(law, q, M, D, F)
+        f2 = _exec_flops_proj(law, q, M, F, D)
+        self.exec_flops = 3 * (f1 + f2)
+        self.dense_flops = 3 * 2 * (2 * M * D * F)
+        self.dominant = aal.AAL_KERNEL_PROJECT
+        self.dominant_flops = f1
+        self.dominant_name = "project (D->F)"
+
+    def config(self):
+        return {"workload": f"{self.name}: {self.law} q={self.q} projections {self.D}->{self.F} and "
+                            f"{self.F}->{self.D}, M={self.M}, fwd + bwd (dX, dW)",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F}
+
+    def bytes_per_set(self):
+        return 2 * (2 * self.D * self.F * 3 + self.M * (self.D + self.F) * 4)
+
+    def setup(self, nsets, seed):
+        self.sets = []
+        a = inputs.projection_inputs(self.M, self.D, self.F, seed=seed, with_dy=True, want_f64=False)
+        b = inputs.projection_inputs(self.M, self.F, self.D, seed=seed + 1, with_dy=True, want_f64=False)
+        for _ in range(nsets):
+            s = {}
+            for tag, ins in (("a", a), ("b", b)):
+                for k in ("X", "W", "dY"):
+                    s[tag + k] = ins[k].t.cuda()
+                s[tag + "Y"] = torch.empty_like(s[tag + "dY"])
+                s[tag + "dX"] = torch.empty_like(s[tag + "X"])
+                s[tag + "dW"] = torch.empty_like(s[tag + "W"])
+            self.sets.append(s)
+        self.rule = aal.row_rule(seq_len=self.seq_len)
+
+    def step(self, i, ev=None):
+        s = self.sets[i % len(self.sets)]
+        if ev is not None:
+            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
+        for t in ("a", "b"):
+            aal.aal_project_fwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "Y"])
+            aal.aal_project_bwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "dY"],
+                                s[t + "dX"], s[t + "dW"])
+
+    def dense_step(self, i):
+        s = self.sets[i % len(self.sets)]
+        for t in ("a", "b"):
+            torch.matmul(s[t + "X"], s[t + "W"], out=s[t + "Y"])
+            torch.matmul(s[t + "dY"], s[t + "W"].t(), out=s[t + "dX"])
+            torch.matmul(s[t + "X"].t(), s[t + "dY"], out=s[t + "dW"])
+
+    e2e_step = None
+
+
+class Square:
+    def __init__(self, name, law, q, n):
+        self.name, self.law, self.q, self.n = name, law, q, n
+        b = n // q
+        self.exec_flops = 2 * aal.aal_block_product_count(law, q, False) * b ** 3
+        self.dense_flops = 2 * n ** 3
+        self.dominant = aal.AAL_KERNEL_SQUARE
+        self.dominant_flops = self.exec_flops
+        self.dominant_name = "square product"
+
+    def config(self):
+        return {"workload": f"{self.name}: square product {self.law} q={self.q} n={self.n} b={self.n // self.q}",
+                "law": self.law, "q": self.q, "n": self.n}
+
+    def bytes_per_set(self):
+        return 3 * self.n * self.n * 2
+
+    def setup(self, nsets, seed):
+        X = torch.randn(self.n, self.n, device="cuda", generator=torch.Generator("cuda").manual_seed(seed)).mul_(
+            self.n ** -0.5).to(torch.bfloat16)
+        W = torch.randn(self.n, self.n, device="cuda", generator=torch.Generator("cuda").manual_seed(seed + 1)).mul_(
+            self.n ** -0.5).to(torch.bfloat16)
+        self.sets = [dict(X=X, W=W, Z=torch.empty_like(X))]
+
+    def step(self, i, ev=None):
+        s = self.sets[0]
+        if ev is not None:
+            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
+        aal.aal_square_product(self.law, self.q, s["X"], s["W"], s["Z"])
+
+    def dense_step(self, i):
+        s = self.sets[0]
+        torch.matmul(s["X"], s["W"], out=s["Z"])
+
+    e2e_step = None
+
+
+WORKLOADS = {
+    "c2": lambda: SwigluDecode("Q2xQ2 110M pilot FFN", "Q2xQ2", 4, 12288, 768, 1536, 1536),
+    "c3": lambda: SwigluDecode("Qwen3-8B-shaped FFN", "Q", 32, 2048, 4096, 12288, 2048,
+                               w_sigma_rule="D", decode_batches=()),
+    "c4": lambda: ProjFwdBwd("Qwen3-30B-A3B-expert-shaped FFN", "Q", 16, 2048, 2048, 768, 2048),
+    "c5": lambda: Square("fixed-block square", "Q", 256, 32768),
+}
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (NVML, read-only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x4: "sw_power_cap", 0x1: "gpu_idle",
+        0x2: "applications_clocks_setting", 0x100: "sync_boost", 0x200: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.01):
+        self.samples, self.reasons, self.period = [], set(), period
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# Timing helpers
+# ---------------------------------------------------------------------------
+
+def _barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def _max_over_ranks(v, dist_on):
+    if not dist_on:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(fn, steps, warmup, dist_on, per_step_events=False):
+    for i in range(warmup):
+        fn(i, None)
+    _barrier(dist_on)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)] if per_step_events else None
+    start.record()
+    for i in range(steps):
+        fn(warmup + i, evs[i] if evs else None)
+    stop.record()
+    _barrier(dist_on)
+    total_ms = start.elapsed_time(stop)
+    kern_ms = [a.elapsed_time(b) for a, b in evs] if evs else None
+    return total_ms, kern_ms
+
+
+def cpu_cores_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return n
+
+
+def run_reference(args, wl):
+    """The oracle on a bounded sample of the workload, on host cores."""
+    rows = args.ref_rows
+    flops, run, desc = wl.oracle_sample(rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    value = flops / dt / 1e12
+    cores = cpu_cores_used()
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": wl.config(),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def cpu_baseline(wl, budget_s, rows):
+    flops, run, desc = wl.oracle_sample(rows)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores_used(), "kind": "oracle",
+            "sample": f"{desc}; {n} run(s), {dt:.3f} s each"}
+
+
+METRIC = "executed BF16 TFLOP/s and % tensor peak per projection; speedup vs dense matmul"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="aal", choices=["aal", "reference"])
+    ap.add_argument("--config", default="c2", choices=sorted(WORKLOADS))
+    ap.add_argument("--sets", type=int, default=0, help="rotating input sets (0: enough to exceed L2)")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=768)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.config]()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    aal.load()
+    peaks = _peaks()
+
+    nsets = args.sets or max(1, min(16, -(-2 * L2_BYTES // max(wl.bytes_per_set(), 1))))
+    wl.setup(nsets, seed=rank)
+
+    # ---- timed region: K steps of the whole path
+    aal.aal_launch_count(reset=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        total_ms, kern_ms = time_steps(lambda i, ev: wl.step(i, ev), args.steps, args.warmup, dist_on,
+                                       per_step_events=True)
+    launches = aal.aal_launch_count(reset=True)
+    launches_timed = launches * args.steps // (args.steps + args.warmup)
+    status = aal.aal_get_device_status()
+    if status != aal.AAL_OK:
+        raise SystemExit(f"device status after the timed region: {aal.status_string(status)}")
+    total_ms = _max_over_ranks(total_ms, dist_on)
+    ms = total_ms / args.steps
+    value = world * wl.exec_flops / (ms * 1e-3) / 1e12
+
+    # ---- dominant kernel: live per-launch CUDA events inside the timed region
+    kms = statistics.mean(kern_ms) if kern_ms else None
+    achieved = wl.dominant_flops / (kms * 1e-3) / 1e12 if kms else None
+    long_region = total_ms > 2000.0
+    peak = peaks["bf16_sust"] if long_region else peaks["bf16"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak if achieved else None, "traffic": None,
+                "kernel": wl.dominant_name, "kernel_ms": kms,
+                "kernel_share_of_step": (kms / ms) if kms else None,
+                "peak_kind": ("sustained" if long_region else "burst") + f" bf16, {peaks['source']}"}
+
+    # ---- dense comparison on the same GPU
+    dense_ms, _ = time_steps(lambda i, ev: wl.dense_step(i), args.steps, args.warmup, dist_on)
+    dense_ms = _max_over_ranks(dense_ms, dist_on) / args.steps
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if wl.e2e_step is not None:
+        e_ms, _ = time_steps(lambda i, ev: wl.e2e_step(i), args.steps, args.warmup, dist_on)
+        e_ms = _max_over_ranks(e_ms, dist_on) / args.steps
+        h2d, d2h = wl.e2e_bytes()
+        e2e = {"value": world * wl.exec_flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    out = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded normal inputs and weights, shapes of the pages' workload)",
+           "config": dict(wl.config(), parallelism=f"token-sharded x{world}, weights replicated",
+                          l2=f"{nsets} rotating input sets of {wl.bytes_per_set() / 2**20:.0f} MiB "
+                             f"(> 126 MiB L2 in total)" if nsets > 1 else "inputs larger than L2"),
+           "tensor_peak_frac": value / world / peak,
+           "dense_ms_per_step": dense_ms, "dense_speedup": dense_ms / ms,
+           "exec_gflop_per_step": wl.exec_flops / 1e9, "dense_gflop_per_step": wl.dense_flops / 1e9,
+           "roofline": roofline, "clocks": clk.summary(), "gpu_launches": launches_timed,
+           "e2e": e2e}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget, args.ref_rows) if hasattr(wl, "oracle_sample") else None
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,237 @@
+/*
+ * libaal — associative-algebra block projections on B200 (sm_100a).
+ *
+ * The operator comes from "Change the Product, Keep the Parameters:
+ * Associative Algebra Layers for Transformers" (Koziev & Oseledets,
+ * arXiv:2609.32814).  A projection Y = X W (X [tokens, din], W [din, dout],
+ * agihunt.info digest, opening paragraph) is cut into q feature groups on
+ * both sides, so W is a q x q grid of blocks W_ak of size (din/q) x (dout/q).
+ * Instead of the row-by-column rule, output block (i, k) of X * W sums only
+ * the products X_ia W_ak with a in S(i, k), where S is the multiplication
+ * table of an associative algebra:
+ *
+ *   complete-graph law Q_q  (agihunt.info digest, multiplication-table
+ *   paragraph): S(i, i) = {i}; S(i, k) = {i, k} for k != i — a diagonal
+ *   block multiplies only its own group, an off-diagonal block is the source
+ *   diagonal times the edge plus the edge times the target diagonal.
+ *   2q^2 - q block products on the square, 2q - 1 per row.
+ *
+ *   tensor-square law Q2 (x) Q2 (agihunt.info digest, tensor-square
+ *   paragraph): 4 groups indexed by pairs g = 2*g1 + g2,
+ *   S((i1,i2),(k1,k2)) = S(i1,k1) x S(i2,k2) under Q_2.  36 block products on
+ *   the square, 9 of 16 per row.
+ *
+ * Row typing (agihunt.info digest, paragraph on the Transformer mapping;
+ * hotpaper.ai summary, "row-typed rectangular projections"): each token gets
+ * a row type t from its absolute position and computes only row t of the
+ * table: y_k = sum_{a in S(t, k)} x_a W_ak.  The type is position mod q.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Matrices are row-major with a leading dimension ``ld`` (elements, >=
+ *   cols).  Every pointer in an aal_mat is DEVICE memory owned by the
+ *   caller; the library never frees or keeps it.
+ * - dtype: AAL_BF16 (bf16 inputs, fp32 accumulation, bf16 outputs) or
+ *   AAL_F32 (fp32 throughout).  All matrices of one call share one dtype.
+ * - The compute calls are asynchronous on ``stream`` (a cudaStream_t; NULL is
+ *   the legacy default stream).  Host-side argument errors are returned
+ *   before anything is launched.  Errors found on the device (an explicit
+ *   row type outside [0, q), a wait that ran out) are recorded in a device
+ *   status word that aal_get_device_status() reads.
+ * - The tensor-core path needs 16-byte aligned base pointers and leading
+ *   dimensions that are multiples of 8 (bf16); other shapes take the general
+ *   CUDA path, which needs 4-byte (fp32) or 2-byte (bf16) alignment only.
+ * - Nothing aborts; no call allocates device memory.
+ */
+#ifndef AAL_H_
+#define AAL_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AAL_API __attribute__((visibility("default")))
+#else
+#define AAL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum aal_status {
+  AAL_OK = 0,
+  AAL_ERR_INVALID_ARG = 1,    /* bad shape, null pointer, unknown enum value */
+  AAL_ERR_UNSUPPORTED = 2,    /* valid request this build cannot serve      */
+  AAL_ERR_ALIGNMENT = 3,      /* pointer / ld misaligned for a required path */
+  AAL_ERR_CUDA = 4,           /* a CUDA runtime call failed                  */
+  AAL_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out             */
+  AAL_ERR_DEVICE_BOUNDS = 6   /* a kernel met an out-of-range index (type)   */
+} aal_status;
+
+typedef enum aal_law {
+  AAL_LAW_Q = 0,     /* complete-graph law Q_q, any q >= 1 */
+  AAL_LAW_Q2XQ2 = 1  /* tensor square Q2 (x) Q2; q must be 4 */
+} aal_law;
+
+typedef enum aal_dtype { AAL_BF16 = 0, AAL_F32 = 1 } aal_dtype;
+
+/* A row-major device matrix: element (r, c) at ((T*)ptr)[r * ld + c]. */
+typedef struct aal_mat {
+  void* ptr;
+  int32_t dtype; /* aal_dtype */
+  int64_t rows;
+  int64_t cols;
+  int64_t ld;
+} aal_mat;
+
+typedef enum aal_row_type_kind {
+  /* Tokens are packed as back-to-back sequences of seq_len tokens; row r sits
+   * at absolute position (r mod seq_len) + pos_offset and has type
+   * position mod q. */
+  AAL_TYPES_POSITION = 0,
+  /* types[r] (device int32 array of length rows) gives row r's type. */
+  AAL_TYPES_EXPLICIT = 1
+} aal_row_type_kind;
+
+typedef struct aal_row_type_rule {
+  int32_t kind;          /* aal_row_type_kind */
+  int64_t seq_len;       /* kind 0: > 0 */
+  int64_t pos_offset;    /* kind 0: >= 0 */
+  const int32_t* types;  /* kind 1: device pointer, not owned */
+} aal_row_type_rule;
+
+/* ---------------------------------------------------------------------- */
+/* Compute calls                                                           */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Row-typed projection Y = X * W (agihunt.info digest, multiplication-table
+ * and Transformer-mapping paragraphs).
+ *   X [M, din], W [din, dout], Y [M, dout]; din and dout divisible by q.
+ *   Row r of type t: Y[r, group k] = sum_{a in S(t,k)} X[r, group a] W_ak.
+ *   Y is overwritten.  M may be 0 (nothing is launched).
+ */
+AAL_API aal_status aal_project_fwd(int32_t law, int32_t q, aal_row_type_rule rule,
+                           aal_mat X, aal_mat W, aal_mat Y, void* stream);
+
+/*
+ * SwiGLU feed-forward block with all three projections algebraic and the same
+ * row types (agihunt.info digest: the pilot changes only the FFN
+ * projections; the full SwiGLU forward is among the measured kernels):
+ *   H = silu(X * Wg) . (X * Wu)   (elementwise; silu(z) = z / (1 + e^-z))
+ *   Y = H * Wd
+ *   X [M, D], Wg and Wu [D, F], Wd [F, D], H [M, F] (caller memory, written
+ *   and kept, e.g. for a backward pass), Y [M, D].
+ *   The SiLU and the product are applied to the fp32 accumulators before H is
+ *   rounded to the call's dtype.
+ */
+AAL_API aal_status aal_swiglu_fwd(int32_t law, int32_t q, aal_row_type_rule rule,
+                          aal_mat X, aal_mat Wg, aal_mat Wu, aal_mat Wd,
+                          aal_mat H, aal_mat Y, void* stream);
+
+/*
+ * Backward of aal_project_fwd for L = <dY, X * W> (agihunt.info digest:
+ * forward plus gradient on the narrow expert FFN shape).
+ *   dX[r, group a] = sum over k with a in S(t_r, k) of dY[r, group k] W_ak^T
+ *   dW_ak          = sum over rows r with a in S(t_r, k) of
+ *                    X[r, group a]^T dY[r, group k]
+ *   dX [M, din] may have ptr == NULL (not computed); likewise dW [din, dout].
+ *   dX is overwritten; dW is overwritten, or added to when accumulate_dW != 0.
+ */
+AAL_API aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rule,
+                           aal_mat X, aal_mat W, aal_mat dY,
+                           aal_mat dX, aal_mat dW, int32_t accumulate_dW,
+                           void* stream);
+
+/*
+ * Decode step: one new token per batch entry (agihunt.info digest: decoding
+ * evaluates only the new position's row, as a matrix-vector product with its
+ * own kernel).
+ *   positions: device int64 array [B], absolute positions (>= 0); the row
+ *   type of entry b is positions[b] mod q.
+ *   x [B, din], W [din, dout], y [B, dout] (overwritten).
+ */
+AAL_API aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* positions,
+                             aal_mat x, aal_mat W, aal_mat y, void* stream);
+
+/*
+ * Full (not row-typed) product of square block matrices, Z = X * W
+ * (agihunt.info digest: fixed-block square product, and the quadratic
+ * arithmetic when the block size stays fixed while q grows).
+ *   X, W, Z [n, n], n divisible by q, block size b = n / q:
+ *   Z_ik = sum_{a in S(i,k)} X_ia W_ak.  Z is overwritten and must not alias
+ *   X or W.
+ */
+AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat W,
+                              aal_mat Z, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Host-side table queries (integer, no GPU needed)                        */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * The multiplication table as the kernels use it: S is HOST memory of q*q*q
+ * bytes, written as S[(i*q + k)*q + a] = 1 if a is in S(i, k), else 0.
+ */
+AAL_API aal_status aal_block_table(int32_t law, int32_t q, uint8_t* S);
+
+/*
+ * Number of block products: row_typed != 0 -> per row type (2q - 1 for Q_q,
+ * 9 for Q2xQ2); row_typed == 0 -> whole square product (2q^2 - q, 36)
+ * (author's post and agihunt.info digest: 6 at q = 2 against 8 dense).
+ * Returns -1 for an invalid law / q.
+ */
+AAL_API int64_t aal_block_product_count(int32_t law, int32_t q, int32_t row_typed);
+
+/* ---------------------------------------------------------------------- */
+/* Status, paths, version                                                  */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Synchronizes ``stream``, then reads and clears the device status word of
+ * the current device: AAL_OK, AAL_ERR_DEVICE_TIMEOUT or
+ * AAL_ERR_DEVICE_BOUNDS (or AAL_ERR_CUDA if the synchronization failed).
+ */
+AAL_API aal_status aal_get_device_status(void* stream);
+
+/* Static English description of a status code (never NULL). */
+AAL_API const char* aal_status_string(int32_t status);
+
+/*
+ * Kernel-path policy for the following calls on this host thread:
+ *   AAL_PATH_AUTO (0): the tensor-core path where the shape allows it, else
+ *   the general CUDA path; AAL_PATH_TENSOR (1): the tensor-core path or
+ *   AAL_ERR_UNSUPPORTED; AAL_PATH_GENERAL (2): always the general CUDA path.
+ * aal_last_path() returns the path the last successful compute call on this
+ * thread launched (1 tensor-core, 2 general, 3 decode kernel, 0 none).
+ */
+enum { AAL_PATH_AUTO = 0, AAL_PATH_TENSOR = 1, AAL_PATH_GENERAL = 2, AAL_PATH_DECODE = 3 };
+AAL_API aal_status aal_set_path_policy(int32_t policy);
+AAL_API int32_t aal_last_path(void);
+
+/*
+ * Optional timing hook for one kernel kind, for the next launch of that kind
+ * on this host thread only: the library records the CUDA event ``before``
+ * (a cudaEvent_t) on the call's stream just before that launch and ``after``
+ * just after it, then forgets both.  Passing NULL events clears the hook.
+ * Kinds: AAL_KERNEL_PROJECT (1, also the down projection inside
+ * aal_swiglu_fwd), AAL_KERNEL_GATE_UP (2, the fused gate/up/SiLU kernel of
+ * aal_swiglu_fwd), AAL_KERNEL_BWD_DX (3), AAL_KERNEL_BWD_DW (4),
+ * AAL_KERNEL_SQUARE (5), AAL_KERNEL_DECODE (6).
+ */
+enum { AAL_KERNEL_PROJECT = 1, AAL_KERNEL_GATE_UP = 2, AAL_KERNEL_BWD_DX = 3,
+       AAL_KERNEL_BWD_DW = 4, AAL_KERNEL_SQUARE = 5, AAL_KERNEL_DECODE = 6 };
+AAL_API aal_status aal_set_timing_events(int32_t kernel, void* before, void* after);
+
+/* Number of kernels launched by compute calls on this thread since the last
+ * reset (for launch accounting). */
+AAL_API int64_t aal_launch_count(int32_t reset);
+
+/* Library version as major*10000 + minor*100 + patch. */
+AAL_API int32_t aal_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AAL_H_ */

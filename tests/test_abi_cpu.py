@@ -1,0 +1,148 @@
+"""CPU-side checks of the C-ABI library: it loads without a GPU, exports every
+symbol include/aal.h declares, its integer table matches the oracle bit for
+bit, and argument errors come back as status codes before any launch."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import associative_algebra_block_b200 as aal
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(aal.LIB_PATH):
+        from associative_algebra_block_b200 import build
+        build.build()
+    return aal.load()
+
+
+def _declared_symbols():
+    names = set()
+    with open(os.path.join(ROOT, "include", "aal.h")) as f:
+        text = f.read()
+    for m in re.finditer(r"^AAL_API\s+[\w\s\*]+?\b(aal_\w+)\s*\(", text, flags=re.M):
+        names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_boundary_calls():
+    names = _declared_symbols()
+    for required in ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd",
+                     "aal_decode_matvec", "aal_square_product", "aal_block_table",
+                     "aal_block_product_count", "aal_get_device_status", "aal_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(aal.EXPORTS) <= _declared_symbols()
+
+
+@pytest.mark.parametrize("law,q", [("Q", 1), ("Q", 2), ("Q", 3), ("Q", 7), ("Q", 16), ("Q", 32),
+                                   ("Q2xQ2", 4)])
+def test_block_table_matches_oracle_bit_exact(lib, law, q):
+    got = aal.aal_block_table(law, q)
+    ref = oracle.block_table_array(law, q)
+    assert got.dtype == ref.dtype and np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("law,q", [("Q", 1), ("Q", 2), ("Q", 5), ("Q", 16), ("Q", 32), ("Q", 256),
+                                   ("Q2xQ2", 4)])
+def test_block_product_counts_match_oracle(lib, law, q):
+    for row_typed in (True, False):
+        assert aal.aal_block_product_count(law, q, row_typed) == oracle.block_product_count(law, q, row_typed)
+
+
+def test_invalid_law_and_q(lib):
+    assert aal.aal_block_product_count("Q2xQ2", 3, True) == -1
+    assert aal.aal_block_product_count(7, 2, True) == -1
+    assert aal.aal_block_product_count("Q", 0, True) == -1
+    S = np.zeros(27, np.uint8)
+    assert lib.aal_block_table(1, 3, S.ctypes.data) == aal.AAL_ERR_INVALID_ARG
+    assert lib.aal_block_table(0, 3, None) == aal.AAL_ERR_INVALID_ARG
+
+
+def _m(ptr, rows, cols, ld=None, dtype=aal.AAL_BF16):
+    return aal.AalMat(ptr, dtype, rows, cols, cols if ld is None else ld)
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("case", ["shape", "q_divides", "null", "ld", "rule", "law", "dtype"])
+def test_project_fwd_argument_errors(lib, case):
+    rule = aal.AalRowTypeRule(0, 64, 0, None)
+    X, W, Y = _m(FAKE, 64, 64), _m(FAKE, 64, 32), _m(FAKE, 64, 32)
+    law, q = 0, 2
+    expect = aal.AAL_ERR_INVALID_ARG
+    if case == "shape":
+        W = _m(FAKE, 32, 32)
+    elif case == "q_divides":
+        q = 3
+    elif case == "null":
+        X = _m(None, 64, 64)
+    elif case == "ld":
+        Y = _m(FAKE, 64, 32, ld=16)
+    elif case == "rule":
+        rule = aal.AalRowTypeRule(0, 0, 0, None)
+    elif case == "law":
+        law = 1
+    elif case == "dtype":
+        Y = _m(FAKE, 64, 32, dtype=aal.AAL_F32)
+        expect = aal.AAL_ERR_UNSUPPORTED
+    assert lib.aal_project_fwd(law, q, rule, X, W, Y, None) == expect
+
+
+def test_other_calls_argument_errors(lib):
+    rule = aal.AalRowTypeRule(0, 16, 0, None)
+    bad_rule = aal.AalRowTypeRule(1, 0, 0, None)
+    X, W = _m(FAKE, 16, 8), _m(FAKE, 8, 8)
+    assert lib.aal_project_fwd(0, 2, bad_rule, X, W, _m(FAKE, 16, 8), None) == aal.AAL_ERR_INVALID_ARG
+    # swiglu: H of the wrong width
+    assert lib.aal_swiglu_fwd(0, 2, rule, X, _m(FAKE, 8, 12), _m(FAKE, 8, 12), _m(FAKE, 12, 8),
+                              _m(FAKE, 16, 8), _m(FAKE, 16, 8), None) == aal.AAL_ERR_INVALID_ARG
+    # bwd: dY of the wrong shape
+    assert lib.aal_project_bwd(0, 2, rule, X, W, _m(FAKE, 16, 4), _m(None, 0, 0), _m(None, 0, 0),
+                               0, None) == aal.AAL_ERR_INVALID_ARG
+    # decode: null positions with rows
+    assert lib.aal_decode_matvec(0, 2, None, _m(FAKE, 4, 8), W, _m(FAKE, 4, 8), None) == aal.AAL_ERR_INVALID_ARG
+    # square: not square / aliasing output
+    assert lib.aal_square_product(0, 2, _m(FAKE, 8, 4), W, _m(FAKE + 4096, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
+    assert lib.aal_square_product(0, 2, X := _m(FAKE, 8, 8), W, _m(FAKE, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
+    # misaligned bf16 pointer
+    assert lib.aal_square_product(0, 2, _m(FAKE + 1, 8, 8), W, _m(FAKE + 4096, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
+
+
+def test_empty_inputs_launch_nothing(lib):
+    rule = aal.AalRowTypeRule(0, 16, 0, None)
+    aal.aal_launch_count(reset=True)
+    assert lib.aal_project_fwd(0, 2, rule, _m(None, 0, 8), _m(FAKE, 8, 8), _m(None, 0, 8), None) == aal.AAL_OK
+    assert lib.aal_square_product(0, 2, _m(None, 0, 0), _m(None, 0, 0), _m(None, 0, 0), None) == aal.AAL_OK
+    assert lib.aal_decode_matvec(0, 2, None, _m(None, 0, 8), _m(FAKE, 8, 8), _m(None, 0, 8), None) == aal.AAL_OK
+    assert aal.aal_launch_count() == 0
+
+
+def test_status_strings(lib):
+    seen = set()
+    for code in range(7):
+        s = aal.aal_status_string(code)
+        assert s and s not in seen
+        seen.add(s)
+    assert aal.aal_status_string(99) == "unknown status"
+
+
+def test_path_policy_round_trip(lib):
+    for p in (aal.AAL_PATH_TENSOR, aal.AAL_PATH_GENERAL, aal.AAL_PATH_AUTO):
+        aal.aal_set_path_policy(p)
+    with pytest.raises(aal.AalError):
+        aal.aal_set_path_policy(7)
+    assert aal.aal_version() >= 100

@@ -1,0 +1,200 @@
+"""GPU parity: every libaal call against the CPU oracle on the same seeded
+inputs.  bf16: max|err|/max|ref| <= 5e-3; fp32: <= 1e-5.  Integer work
+(associativity and unit on small-integer matrices) is compared bit for bit."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import associative_algebra_block_b200 as aal
+from associative_algebra_block_b200 import inputs
+
+from gpu_cases import TOL, host64, run_bwd, run_decode, run_project, run_square, run_swiglu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    aal.load()
+
+
+GENERAL = aal.AAL_PATH_GENERAL
+
+# ----------------------------------------------------------------- Q_2 fp32
+def test_c1_q2_fp32_projection():
+    err, _ = run_project("Q", 2, 64, 64, 64, "f32", seq_len=64)
+    assert err <= TOL["f32"], err
+
+
+@pytest.mark.parametrize("law,q,n", [("Q", 2, 32), ("Q", 3, 48), ("Q2xQ2", 4, 64)])
+def test_c1_integer_associativity_and_unit_exact(law, q, n):
+    mats = inputs.integer_square_inputs(n, count=3, seed=q)
+    X, W, Z = (m.t.cuda() for m in mats)
+
+    def sq(A, B):
+        out = torch.empty_like(A)
+        aal.aal_square_product(law, q, A, B, out)
+        return out
+
+    left = sq(sq(X, W), Z)
+    right = sq(X, sq(W, Z))
+    torch.cuda.synchronize()
+    assert torch.equal(left, right)
+    ref = oracle.square_product(law, q, oracle.square_product(law, q, mats[0].f64, mats[1].f64), mats[2].f64)
+    assert np.array_equal(host64(left), ref)
+    one = torch.eye(n, device="cuda")
+    assert torch.equal(sq(X, one), X) and torch.equal(sq(one, X), X)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_c1_all_calls_small(dtype):
+    tol = TOL[dtype]
+    e, _ = run_square("Q", 2, 64, dtype)
+    assert e <= tol
+    eh, ey, _ = run_swiglu("Q", 2, 64, 64, 128, dtype, seq_len=64)
+    assert eh <= tol and ey <= tol
+    edx, edw, _ = run_bwd("Q", 2, 64, 64, 64, dtype)
+    assert edx <= tol and edw <= tol
+    ed, _ = run_decode("Q", 2, 5, 64, 64, dtype)
+    assert ed <= tol
+
+
+# ------------------------------------------------- Q2 x Q2 SwiGLU (110M FFN)
+def test_c2_swiglu_full_size():
+    eh, ey, path = run_swiglu("Q2xQ2", 4, 12288, 768, 1536, "bf16", seq_len=1536)
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+
+
+@pytest.mark.parametrize("B", [1, 8, 64])
+def test_c2_decode(B):
+    err, path = run_decode("Q2xQ2", 4, B, 768, 1536, "bf16", seed=B)
+    assert err <= TOL["bf16"], err
+    assert path == aal.AAL_PATH_DECODE
+    err, _ = run_decode("Q2xQ2", 4, B, 1536, 768, "bf16", seed=B + 1)
+    assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("t", [0, 1, 2, 3])
+def test_c2_decode_single_type(t):
+    err, _ = run_decode("Q2xQ2", 4, 1, 768, 1536, "bf16", seed=40 + t, same_type=t)
+    assert err <= TOL["bf16"], err
+
+
+# -------------------------------------------------- Qwen3-8B-shaped Q_32
+def test_c3_swiglu_full_size():
+    eh, ey, path = run_swiglu("Q", 32, 2048, 4096, 12288, "bf16", seq_len=2048, w_sigma_rule="D")
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+
+
+# ------------------------------------------ Qwen3-30B-A3B-expert-shaped Q_16
+@pytest.mark.parametrize("din,dout", [(2048, 768), (768, 2048)])
+def test_c4_projection_fwd_bwd(din, dout):
+    err, _ = run_project("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
+    assert err <= TOL["bf16"], err
+    edx, edw, _ = run_bwd("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
+    assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
+
+
+def test_c4_swiglu():
+    eh, ey, _ = run_swiglu("Q", 16, 2048, 2048, 768, "bf16", seq_len=2048)
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+
+
+# ------------------------------------------------- square product Q_256
+def test_c5_square_full_size_sampled_tiles():
+    n, q = 32768, 256
+    b = n // q
+    ins = inputs.square_inputs(n, seed=0, dtype="bf16", want_f64=False)
+    X, W = ins["X"].t.cuda(), ins["W"].t.cuda()
+    Z = torch.empty_like(X)
+    aal.aal_square_product("Q", q, X, W, Z)
+    torch.cuda.synchronize()
+    Xh, Wh = ins["X"].t, ins["W"].t
+    rng = np.random.default_rng(123)
+    tiles = [(0, 0), (0, q - 1), (q - 1, 0), (q - 1, q - 1), (17, 17), (5, 200)]
+    tiles += [tuple(int(v) for v in rng.integers(0, q, 2)) for _ in range(26)]
+
+    def blk(A, r, c):
+        return A[r * b:(r + 1) * b, c * b:(c + 1) * b].to(torch.float64).numpy()
+
+    worst = 0.0
+    for i, k in tiles:
+        ref = oracle.square_tile("Q", q, i, k, lambda r, c: blk(Xh, r, c), lambda r, c: blk(Wh, r, c))
+        got = Z[i * b:(i + 1) * b, k * b:(k + 1) * b].to("cpu", torch.float64).numpy()
+        worst = max(worst, oracle.rel_err(got, ref))
+    assert worst <= TOL["bf16"], worst
+
+
+@pytest.mark.parametrize("law,q,n", [("Q", 4, 512), ("Q", 16, 2048), ("Q2xQ2", 4, 256)])
+def test_square_medium(law, q, n):
+    err, _ = run_square(law, q, n, "bf16")
+    assert err <= TOL["bf16"], err
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("M", [0, 1, 7, 130, 1000])
+def test_ragged_and_empty_rows(M):
+    for law, q, din, dout in (("Q", 4, 256, 512), ("Q2xQ2", 4, 256, 128)):
+        if M == 0:
+            X = torch.empty(0, din, dtype=torch.bfloat16, device="cuda")
+            W = torch.randn(din, dout, device="cuda").to(torch.bfloat16)
+            Y = torch.empty(0, dout, dtype=torch.bfloat16, device="cuda")
+            aal.aal_project_fwd(law, q, aal.row_rule(seq_len=16), X, W, Y)
+            continue
+        err, _ = run_project(law, q, M, din, dout, "bf16", seq_len=M)
+        assert err <= TOL["bf16"], (law, M, err)
+
+
+@pytest.mark.parametrize("seq_len,offset", [(100, 0), (64, 3), (1536, 0), (37, 11)])
+def test_sequence_packing_and_offset(seq_len, offset):
+    err, _ = run_project("Q", 8, 600, 256, 256, "bf16", seq_len=seq_len, offset=offset)
+    assert err <= TOL["bf16"], err
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_explicit_types(dtype):
+    err, _ = run_project("Q", 8, 333, 128, 256, dtype, explicit=True)
+    assert err <= TOL[dtype], err
+    edx, edw, _ = run_bwd("Q", 8, 333, 128, 256, dtype, explicit=True)
+    assert edx <= TOL[dtype] and edw <= TOL[dtype]
+
+
+def test_q1_is_dense():
+    err, _ = run_project("Q", 1, 256, 128, 192, "bf16", seq_len=256)
+    assert err <= TOL["bf16"], err
+
+
+def test_bwd_accumulate():
+    edx, edw, _ = run_bwd("Q", 4, 512, 256, 256, "bf16", accumulate=True)
+    assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
+
+
+def test_general_path_matches_oracle():
+    err, path = run_project("Q", 16, 2048, 2048, 768, "bf16", seq_len=2048, policy=GENERAL)
+    assert err <= TOL["bf16"] and path == aal.AAL_PATH_GENERAL
+
+
+def test_out_of_range_explicit_type_sets_device_status():
+    q, M, din, dout = 4, 64, 64, 64
+    X = torch.randn(M, din, device="cuda").to(torch.bfloat16)
+    W = torch.randn(din, dout, device="cuda").to(torch.bfloat16)
+    Y = torch.zeros(M, dout, dtype=torch.bfloat16, device="cuda")
+    types = torch.zeros(M, dtype=torch.int32, device="cuda")
+    types[5] = 9
+    aal.aal_project_fwd("Q", q, aal.row_rule(types=types), X, W, Y)
+    assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
+    assert aal.aal_get_device_status() == aal.AAL_OK  # cleared by the read
+    assert torch.all(Y[5] == 0)
+
+
+def test_negative_decode_position_sets_device_status():
+    x = torch.randn(2, 64, device="cuda").to(torch.bfloat16)
+    W = torch.randn(64, 64, device="cuda").to(torch.bfloat16)
+    y = torch.zeros(2, 64, dtype=torch.bfloat16, device="cuda")
+    aal.aal_decode_matvec("Q", 2, torch.tensor([3, -1], device="cuda"), x, W, y)
+    assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
