@@ -148,9 +148,16 @@ def row_rule(seq_len: int | None = None, pos_offset: int = 0,
     return AalRowTypeRule(AAL_TYPES_POSITION, int(seq_len), int(pos_offset), None)
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream) -> int | None:
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+        if not torch.cuda.is_available():
+            return None
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
+        return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)

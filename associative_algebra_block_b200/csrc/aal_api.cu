@@ -15,13 +15,23 @@ void note_path(int path) { t_last_path = path; }
 static thread_local cudaEvent_t t_ev_before[8] = {};
 static thread_local cudaEvent_t t_ev_after[8] = {};
 
+// Records an event on ``s``; while ``s`` is being captured into a CUDA graph
+// the record becomes an event-record node, so the event still timestamps the
+// launch each time the graph runs.
+static cudaError_t record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return cudaErrorUnknown;
+  if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  return cudaEventRecord(e, s);
+}
+
 // Records the one-shot timing events of ``kind`` around ``launch``.
 template <typename F>
 static aal_status timed(int kind, cudaStream_t s, F launch) {
   cudaEvent_t b = t_ev_before[kind], a = t_ev_after[kind];
-  if (b && cudaEventRecord(b, s) != cudaSuccess) return AAL_ERR_CUDA;
+  if (b && record_event(b, s) != cudaSuccess) return AAL_ERR_CUDA;
   aal_status st = launch();
-  if (a && st == AAL_OK && cudaEventRecord(a, s) != cudaSuccess) return AAL_ERR_CUDA;
+  if (a && st == AAL_OK && record_event(a, s) != cudaSuccess) return AAL_ERR_CUDA;
   if (st == AAL_OK) { t_ev_before[kind] = nullptr; t_ev_after[kind] = nullptr; }
   return st;
 }

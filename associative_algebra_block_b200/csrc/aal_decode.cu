@@ -3,12 +3,20 @@
 // position's row, as a matrix-vector product with a kernel of its own).
 //
 // The work is a stream over the weight rows that some entry of the batch
-// needs.  A CTA owns a 64-column slab of W and a tile of up to kDecodeBT batch
-// entries; its 8 warps split the weight rows, every lane owns two adjacent
-// columns, and the warps' partial sums meet in shared memory.  A weight row is
-// loaded only when some entry of the tile needs its group for one of the
-// lane's columns, so one row type touches (2q-1)/q^2 of W (9/16 for Q2xQ2).
+// needs: a weight row is loaded only when some entry of a CTA's batch tile
+// needs its group for the thread's columns, so one row type touches
+// (2q-1)/q^2 of W (9/16 for Q2xQ2) in arithmetic.  k_decode_split (weight
+// rows split across a thread-block cluster, activations staged in shared
+// memory) serves aligned bf16 weights whose output groups are multiples of
+// 64 columns; k_decode_vec (16-byte vector loads, rows loaded only when some
+// entry needs them) the other aligned ones, fp32 included; k_decode is the
+// scalar fallback.
+#include <cooperative_groups.h>
+#include <limits.h>
+
 #include "aal_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace aal {
 
@@ -102,12 +110,403 @@ k_decode(int law, int q, const int64_t* __restrict__ pos, long long B, const T* 
   }
 }
 
+// Vectorised variant: every thread owns VEC adjacent columns (16 bytes of a
+// weight row) and, per pass, keeps up to kRP independent 16-byte weight loads
+// in flight before consuming them, so the stream is bandwidth- rather than
+// latency-bound.  Thread (cv, rl): cv picks the column vector (4 per CTA), rl
+// the row lane (64 per CTA, rows rl, rl + 64, ...).  Partial sums over the row
+// lanes meet first through warp shuffles (8 row lanes per warp), then through
+// shared memory (8 warps).
+constexpr int kVecBB = 8;  // batch entries per CTA
+constexpr int kRP = 8;     // weight rows per thread per pass
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4& u, float* f) {
+  f[0] = __uint_as_float(u.x);
+  f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z);
+  f[3] = __uint_as_float(u.w);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_decode_vec(int law, int q, const int64_t* __restrict__ pos, int B, const T* __restrict__ x,
+             long long ldx, const T* __restrict__ W, long long ldw, T* __restrict__ y,
+             long long ldy, int bi, int bo, int din, int dout) {
+  constexpr int VEC = 16 / sizeof(T);
+  constexpr int CW = 4 * VEC;  // columns per CTA
+  __shared__ int s_type[kVecBB];
+  __shared__ float red[8][kVecBB][CW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cv = lane & 3, rl = warp * 8 + (lane >> 2);
+  const int col = blockIdx.x * CW + cv * VEC;
+  const bool cvalid = col < dout;
+  const int k = cvalid ? col / bo : 0;
+  const int b0 = blockIdx.y * kVecBB;
+
+  if (threadIdx.x < kVecBB) {
+    int t = -1;
+    const int b = b0 + threadIdx.x;
+    if (b < B) {
+      const long long p = pos[b];
+      if (p < 0) flag_device_error(kDevBounds);
+      else t = (int)(p % q);
+    }
+    s_type[threadIdx.x] = t;
+  }
+  __syncthreads();
+  int types[kVecBB];
+#pragma unroll
+  for (int b = 0; b < kVecBB; ++b) types[b] = s_type[b];
+
+  float acc[kVecBB][VEC];
+#pragma unroll
+  for (int b = 0; b < kVecBB; ++b)
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) acc[b][c] = 0.f;
+
+  for (int j0 = 0; j0 < din; j0 += 64 * kRP) {
+    uint4 wv[kRP];
+    unsigned use[kRP];  // bit b: entry b of the tile needs this row
+#pragma unroll
+    for (int i = 0; i < kRP; ++i) {
+      const int j = j0 + rl + 64 * i;
+      unsigned m = 0;
+      if (cvalid && j < din) {
+        const int a = j / bi;
+#pragma unroll
+        for (int b = 0; b < kVecBB; ++b)
+          if (types[b] >= 0 && in_table(law, types[b], k, a)) m |= 1u << b;
+      }
+      use[i] = m;
+      if (m) wv[i] = __ldg(reinterpret_cast<const uint4*>(W + (long long)j * ldw + col));
+    }
+    float w[kRP][VEC];
+#pragma unroll
+    for (int i = 0; i < kRP; ++i) {
+      if (use[i]) unpack16<T>(wv[i], w[i]);
+      else
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) w[i][c] = 0.f;
+    }
+    // one batch entry at a time: its kRP activations are independent loads
+#pragma unroll
+    for (int b = 0; b < kVecBB; ++b) {
+      float xv[kRP];
+#pragma unroll
+      for (int i = 0; i < kRP; ++i) {
+        const int j = j0 + rl + 64 * i;
+        xv[i] = (use[i] >> b & 1u) ? dec_ld(x + (long long)(b0 + b) * ldx + j) : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kRP; ++i)
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) acc[b][c] = fmaf(xv[i], w[i][c], acc[b][c]);
+    }
+  }
+  // reduce over the 8 row lanes of this warp (lane bits 2..4)
+#pragma unroll
+  for (int b = 0; b < kVecBB; ++b)
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) {
+      float v = acc[b][c];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[b][c] = v;
+    }
+  if ((lane >> 2) == 0) {
+#pragma unroll
+    for (int b = 0; b < kVecBB; ++b)
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) red[warp][b][cv * VEC + c] = acc[b][c];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kVecBB * CW; e += blockDim.x) {
+    const int b = e / CW, cc = e % CW;
+    const int c = blockIdx.x * CW + cc;
+    if (b0 + b >= B || c >= dout || s_type[b] < 0) continue;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[w][b][cc];
+    dec_st(y + (long long)(b0 + b) * ldy + c, sum);
+  }
+}
+
+// Split-K cluster variant (the default for aligned bf16 weights).  A
+// thread-block cluster of CL CTAs shares one 64-column slab (inside one output
+// group k) and one tile of TB batch entries; CTA z of the cluster streams
+// weight rows [z*R, (z+1)*R).
+//  - The batch is ranked by row type (ties by index) so that a tile, and the
+//    NB entries of one thread, mostly share a type; a thread skips the rows
+//    none of its entries needs, so arithmetic follows (2q-1)/q^2 of W.
+//  - The first round of weight loads is issued before anything else.
+//  - Activations are staged once with 16-byte loads, already masked by the
+//    table (x[b][j] = 0 unless the group of j is in S(t_b, k)) and widened to
+//    fp32.
+//  - Partial sums meet through warp shuffles and shared memory; across the
+//    cluster every CTA finalises an equal share of the outputs, reading its
+//    peers' partial sums through distributed shared memory.
+// Thread layout: cv = lane & 7 picks 8 columns; the 32 slots (warp, lane>>3)
+// are split into BL batch lanes x RL row lanes; a thread owns NB entries.
+constexpr int kMaxRowsCta = 192;  // multiple of 8
+constexpr int kRound = 8;       // weight rows per thread per round
+constexpr int kRankMax = 256;   // batches up to this size are ranked by type
+
+template <int NB, int RL>
+__global__ void __launch_bounds__(256)
+k_decode_split(int law, int q, const int64_t* __restrict__ pos, int B,
+               const __nv_bfloat16* __restrict__ x, long long ldx,
+               const __nv_bfloat16* __restrict__ W, long long ldw, __nv_bfloat16* __restrict__ y,
+               long long ldy, int bi, int bo, int din, int rows_per_cta) {
+  constexpr int BL = 32 / RL;
+  constexpr int TB = NB * BL;  // batch entries per CTA
+  constexpr int CW = 64;
+  __shared__ __align__(16) float xs[TB][kMaxRowsCta];  // masked fp32 activations
+  __shared__ float red[RL == 32 ? 8 : 1][TB][CW];
+  __shared__ int s_type[TB];
+  __shared__ int s_idx[TB];
+  __shared__ int s_tall[kRankMax];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cv = lane & 7, slot = warp * 4 + (lane >> 3);
+  const int rl = slot % RL, bl = slot / RL;
+  const int col0 = blockIdx.x * CW, col = col0 + cv * 8;
+  const int k = col0 / bo;
+  const int y0 = blockIdx.y * TB;
+  const int r0 = blockIdx.z * rows_per_cta;
+  const int r1 = min(din, r0 + rows_per_cta);
+  const int R = r1 - r0;
+  // 1. first round of weight rows, unconditionally
+  uint4 wv[kRound];
+#pragma unroll
+  for (int u = 0; u < kRound; ++u) {
+    const int j = r0 + rl + RL * u;
+    if (j < r1) wv[u] = __ldg(reinterpret_cast<const uint4*>(W + (long long)j * ldw + col));
+  }
+  // 2. row types; the tile = entries of rank y0 .. y0+TB-1 in type order
+  const bool ranked = B <= kRankMax;
+  if (ranked) {
+    for (int b = tid; b < B; b += blockDim.x) {
+      const long long p = pos[b];
+      s_tall[b] = p < 0 ? q : (int)(p % q);  // invalid positions sort last
+    }
+    __syncthreads();
+    for (int b = tid; b < B; b += blockDim.x) {
+      const int t = s_tall[b];
+      int r = 0;
+      for (int c = 0; c < B; ++c) {
+        const int u = s_tall[c];
+        r += (u < t) || (u == t && c < b);
+      }
+      if (r >= y0 && r < y0 + TB) {
+        s_idx[r - y0] = b;
+        s_type[r - y0] = t < q ? t : -1;
+        if (t >= q && blockIdx.x == 0 && blockIdx.z == 0) flag_device_error(kDevBounds);
+      }
+    }
+    if (tid < TB && y0 + tid >= B) { s_idx[tid] = 0; s_type[tid] = -1; }
+  } else if (tid < TB) {
+    int t = -1;
+    const int b = y0 + tid;
+    if (b < B) {
+      const long long p = pos[b];
+      if (p < 0) { if (blockIdx.x == 0 && blockIdx.z == 0) flag_device_error(kDevBounds); }
+      else t = (int)(p % q);
+    }
+    s_idx[tid] = b < B ? b : 0;
+    s_type[tid] = t;
+  }
+  __syncthreads();
+
+  // 3. masked, widened activations of this CTA's rows (16-byte loads; rows
+  // of entries outside the batch stay unread)
+  const int nvec = R >> 3;  // R is a multiple of 8 when this kernel runs
+  const int nvalid = min(TB, B - y0);
+  for (int e = tid; e < TB * nvec; e += blockDim.x) {
+    const int i = e / nvec, v8 = e - i * nvec, jj = v8 * 8, j = r0 + jj;
+    const int t = i < nvalid ? s_type[i] : -1;
+    float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (t >= 0) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (long long)s_idx[i] * ldx + j));
+      unpack16<__nv_bfloat16>(u, f);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (!in_table(law, t, k, (j + m) / bi)) f[m] = 0.f;
+    }
+    float4* d = reinterpret_cast<float4*>(&xs[i][jj]);
+    d[0] = make_float4(f[0], f[1], f[2], f[3]);
+    d[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+  __syncthreads();
+
+  int types[NB];
+#pragma unroll
+  for (int n = 0; n < NB; ++n) types[n] = s_type[bl * NB + n];
+  float acc[NB][8];
+#pragma unroll
+  for (int n = 0; n < NB; ++n)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[n][c] = 0.f;
+
+  for (int jr = r0 + rl; jr < r1; jr += RL * kRound) {
+    uint4 nxt[kRound];
+    const int jn = jr + RL * kRound;
+#pragma unroll
+    for (int u = 0; u < kRound; ++u) {  // next round in flight while this one computes
+      const int j = jn + RL * u;
+      if (j < r1) nxt[u] = __ldg(reinterpret_cast<const uint4*>(W + (long long)j * ldw + col));
+    }
+#pragma unroll
+    for (int u = 0; u < kRound; ++u) {
+      const int j = jr + RL * u;
+      if (j >= r1) continue;
+      const int a = j / bi;
+      bool need = false;
+#pragma unroll
+      for (int n = 0; n < NB; ++n) need |= types[n] >= 0 && in_table(law, types[n], k, a);
+      if (!need) continue;
+      float w[8];
+      unpack16<__nv_bfloat16>(wv[u], w);
+#pragma unroll
+      for (int n = 0; n < NB; ++n) {
+        const float xv = xs[bl * NB + n][j - r0];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[n][c] = fmaf(xv, w[c], acc[n][c]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kRound; ++u) wv[u] = nxt[u];
+  }
+
+  // 5. reduce over the row lanes: shuffles over lane bits 3..4, then warps
+#pragma unroll
+  for (int n = 0; n < NB; ++n)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v = acc[n][c];
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      acc[n][c] = v;
+    }
+  const float* part;
+  if constexpr (RL == 32) {
+    if ((lane >> 3) == 0) {
+#pragma unroll
+      for (int n = 0; n < NB; ++n)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[warp][n][cv * 8 + c] = acc[n][c];
+    }
+    __syncthreads();
+    for (int e = tid; e < TB * CW; e += blockDim.x) {
+      const int b = e / CW, cc = e % CW;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sum += red[w][b][cc];
+      red[0][b][cc] = sum;
+    }
+    part = &red[0][0][0];
+  } else {  // RL == 4: each warp holds distinct entries after the shuffles
+    if ((lane >> 3) == 0) {
+#pragma unroll
+      for (int n = 0; n < NB; ++n)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[0][bl * NB + n][cv * 8 + c] = acc[n][c];
+    }
+    part = &red[0][0][0];
+  }
+  __syncthreads();
+
+  // 4. across the cluster: CTA r sums outputs r, r + CL, ... of every CTA's
+  // partials through distributed shared memory and writes them
+  cluster.sync();
+  const int cl = (int)cluster.num_blocks(), me = (int)cluster.block_rank();
+  for (int e = me * blockDim.x + tid; e < TB * CW; e += cl * blockDim.x) {
+    const int b = e / CW, cc = e % CW;
+    if (y0 + b >= B || s_type[b] < 0) continue;
+    float sum = 0.f;
+    for (int r = 0; r < cl; ++r) sum += *cluster.map_shared_rank(part + e, r);
+    y[(long long)s_idx[b] * ldy + col0 + cc] = __float2bfloat16_rn(sum);
+  }
+  cluster.sync();  // peers keep their shared memory until every CTA has read it
+}
+
+template <int NB, int RL>
+static cudaError_t launch_split(const cudaLaunchConfig_t& cfg0, int cl, int law, int q,
+                                const int64_t* positions, int B, const aal_mat& x,
+                                const aal_mat& W, const aal_mat& y, int bi, int bo, int rows) {
+  cudaLaunchConfig_t cfg = cfg0;
+  constexpr int TB = NB * (32 / RL);
+  cfg.gridDim.y = (unsigned)((B + TB - 1) / TB);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = cl;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_decode_split<NB, RL>, law, q, positions, B,
+                            (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr, W.ld,
+                            (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)x.cols, rows);
+}
+
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
                          const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled) {
   *handled = true;
   const long long B = x.rows, dout = W.cols;
   if (B == 0 || dout == 0) return AAL_OK;
   const int bi = (int)(x.cols / q), bo = (int)(dout / q);
+  const int es = x.dtype == AAL_F32 ? 4 : 2, vec = 16 / es;
+  const bool vec_ok = ((uintptr_t)W.ptr % 16) == 0 && W.ld % vec == 0 && bo % vec == 0 &&
+                      x.cols <= INT_MAX && dout <= INT_MAX && B <= INT_MAX;
+  // fp32 stays on the exact vector path below
+  if (vec_ok && x.dtype == AAL_BF16 && bo % 64 == 0) {
+    int cl = 1;
+    while (cl < 8 && (x.cols + cl - 1) / cl > kMaxRowsCta) cl <<= 1;
+    while (cl < 8 && (x.cols + cl - 1) / cl > 96) cl <<= 1;  // shorter row ranges
+    const int rows = (int)(((x.cols + cl - 1) / cl + 7) / 8 * 8);
+    if (rows <= kMaxRowsCta && x.cols % 8 == 0 && x.ld % 8 == 0 && ((uintptr_t)x.ptr % 16) == 0 &&
+        (B + 7) / 8 <= 65535) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(dout / 64), 1, (unsigned)cl);
+      cfg.blockDim = dim3(256);
+      cfg.stream = s;
+      const cudaError_t e =
+          B <= 8 ? launch_split<8, 32>(cfg, cl, law, q, positions, (int)B, x, W, y, bi, bo, rows)
+                 : launch_split<4, 4>(cfg, cl, law, q, positions, (int)B, x, W, y, bi, bo, rows);
+      note_launch();
+      return cuda_status(e);
+    }
+  }
+  if (vec_ok) {
+    dim3 grd((unsigned)((dout + 4 * vec - 1) / (4 * vec)), (unsigned)((B + kVecBB - 1) / kVecBB));
+    if (grd.y <= 65535) {
+      if (x.dtype == AAL_F32)
+        k_decode_vec<float><<<grd, 256, 0, s>>>(law, q, positions, (int)B, (const float*)x.ptr,
+                                                x.ld, (const float*)W.ptr, W.ld, (float*)y.ptr,
+                                                y.ld, bi, bo, (int)x.cols, (int)dout);
+      else
+        k_decode_vec<__nv_bfloat16><<<grd, 256, 0, s>>>(
+            law, q, positions, (int)B, (const __nv_bfloat16*)x.ptr, x.ld,
+            (const __nv_bfloat16*)W.ptr, W.ld, (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)x.cols,
+            (int)dout);
+      note_launch();
+      return cuda_status(cudaGetLastError());
+    }
+  }
   dim3 grd((unsigned)((dout + kDecodeCols - 1) / kDecodeCols),
            (unsigned)((B + kDecodeBT - 1) / kDecodeBT));
   if (grd.y > 65535) { *handled = false; return AAL_ERR_UNSUPPORTED; }

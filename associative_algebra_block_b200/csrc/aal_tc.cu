@@ -1,20 +1,1337 @@
-// Tensor-core path (tcgen05 / TMEM / TMA) — filled in below.
+// Tensor-core path: one persistent, warp-specialised tcgen05 kernel for every
+// block product of the algebra.
+//
+// What it computes.  Every call is a set of output tiles; a tile is a
+// 128 x N fp32 accumulator in tensor memory (TMEM) that sums, over the
+// members a of a table entry S(t, k), the block products X_a W_ak (agihunt.info
+// digest, multiplication-table paragraph).  The K range of a tile is a list of
+// up to four "segments" (one per table member, or a merged contiguous range),
+// walked in 64-element chunks; each chunk is one TMA load of an A tile and a B
+// tile into shared memory and up to four tcgen05.mma instructions (K = 16
+// each) accumulating into TMEM.  Because the |S| products of a tile land in
+// the same accumulator, the sum over the table never round-trips through HBM.
+//
+// Row typing without a gather pass.  A token of type t sits at rows
+// r = j*q + c with c = (t - offset) mod q when sequences are multiples of q
+// long (agihunt.info digest: the type comes from the absolute position).  A
+// row-major [M, d] matrix is therefore described to TMA as a 3-D tensor
+// [M/q][q][d]; a box with extent 1 in the middle dimension pulls the rows of
+// one type class straight out of HBM.  No index buffer, no copy.
+//
+// Roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
+// the MMAs (one thread), warps 2..9 drain TMEM to registers and write bf16
+// results (optionally applying SiLU(g)*u or adding into the destination); two
+// epilogue warps share each 32-lane quarter of TMEM and split its columns.
+// Tiles are visited longest first: a tile's cost is the number of block
+// products in its table entry (1, 2 or 4 for the laws here, up to q for the
+// backward's diagonal blocks), and the persistent CTAs stride through the
+// cost-sorted list so that every CTA ends with the short tiles.
+// Shared-memory stages and the two TMEM accumulator buffers are handed over
+// with mbarriers; every wait is bounded (2 s of global time) and on expiry the
+// kernel records AAL_ERR_DEVICE_TIMEOUT in the status word, lets in-flight
+// copies and MMAs land, frees TMEM and returns.
+#include <cuda.h>
+#include <limits.h>
+#include <stdlib.h>
+
 #include "aal_internal.h"
 
 namespace aal {
+namespace tc {
 
-aal_status tc_project(int, int, const RowTypes&, long long, const aal_mat&, const aal_mat&,
-                      const aal_mat&, cudaStream_t) { return AAL_ERR_UNSUPPORTED; }
-aal_status tc_swiglu_gate_up(int, int, const RowTypes&, long long, const aal_mat&, const aal_mat&,
-                             const aal_mat&, const aal_mat&, cudaStream_t) {
-  return AAL_ERR_UNSUPPORTED;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kMaxPairs = 256;
+constexpr int kMaxStages = 8;
+constexpr int kSmemBudget = 200 * 1024;
+constexpr int kEpiSmem = kEpiWarps * 2048;  // TMA-store staging
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+enum Op : int { OP_FWD = 0, OP_SWIGLU = 1, OP_DX = 2, OP_DW = 3, OP_SQUARE = 4 };
+
+// Exact unsigned division by a runtime constant (x < 2^31): q = (hi(x*m) + x) >> s.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+__host__ __device__ inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.s = 0;
+  while ((1u << f.s) < d) ++f.s;
+  f.m = (uint32_t)((((uint64_t)1 << 32) * (((uint64_t)1 << f.s) - d)) / d + 1);
+  return f;
 }
-aal_status tc_project_bwd_dx(int, int, const RowTypes&, long long, const aal_mat&, const aal_mat&,
-                             const aal_mat&, cudaStream_t) { return AAL_ERR_UNSUPPORTED; }
-aal_status tc_project_bwd_dw(int, int, const RowTypes&, long long, const aal_mat&, const aal_mat&,
-                             const aal_mat&, int, cudaStream_t) { return AAL_ERR_UNSUPPORTED; }
-aal_status tc_square(int, int, const aal_mat&, const aal_mat&, const aal_mat&, cudaStream_t) {
-  return AAL_ERR_UNSUPPORTED;
+__device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) {
+  return (uint32_t)(((uint64_t)__umulhi(x, f.m) + x) >> f.s);
+}
+
+struct Seg {
+  int k0;   // first K index of the segment (feature column, or token within the class)
+  int len;  // K extent
+  int cls;  // row class used for coordinate 1 of gathered operands
+  int map;  // which of the two maps of a gathered operand (dW: 1 = contiguous rows)
+};
+
+struct Params {
+  CUtensorMap mapA[2];
+  CUtensorMap mapB[2];
+  CUtensorMap mapOut;  // output seen as [rows/qv][qv][cols]: box {16, 1, 32} (SW32)
+                       // or, when swapped, {32, 1, 16} (no swizzle)
+  int op, law, q, off;
+  int bi, bo;          // block sizes of the two grouped dimensions (op specific)
+  int n_mma;           // MMA N (the MMA M is always 128)
+  int a_aw, b_aw;      // atom width (elements) of MN-major A / B tiles: 64 or 16
+  int a_rows, b_rows;  // MN extent of the A tile (128) and of the B tile (n_mma)
+  int swap;            // 1: TMEM lanes run along the column side of the output
+  int n1, n2, n3;      // tile index = ((i0*n1 + i1)*n2 + i2)*n3 + i3
+  int ntiles;
+  long long Mq;        // rows per class of gathered operands
+  long long Mall;      // all rows (dW over a contiguous map)
+  int qv;              // classes in the gathered view
+  int xr;              // token rows per tile
+  int wn;              // output columns per tile on the weight side
+  uint32_t idesc;      // tcgen05 instruction descriptor (kind::f16, bf16 x bf16 -> f32)
+  uint32_t idesc2;     // same with N = 2 * n_mma (gate and up tiles read as one operand)
+  int fuse_b;          // DUAL == 1: issue one MMA over both B tiles
+  int stages;
+  uint32_t stage_bytes, a_bytes, b_bytes;
+  int acc_cols;        // TMEM columns of one accumulator set
+  uint32_t tmem_cols;  // TMEM allocation (power of two)
+  int swiglu;          // epilogue: silu(acc0) * acc1
+  int accumulate;      // epilogue: out += acc (register path, no TMA store)
+  int tma_store;       // epilogue: stage in shared memory and store with TMA
+  __nv_bfloat16* out;
+  long long ldo;
+  // Tile order: pair rank -> (p0, p1).  For q <= 16 the host stores the pairs
+  // sorted by cost (p0 << 8 | p1); otherwise the law is Q_q and the diagonal
+  // pairs go first (diag_first) or last.
+  int npairs_list;
+  int diag_first;
+  uint16_t pairs[kMaxPairs];
+  FastDiv div_n1, div_n3, div_qm1;
+  int a_merged, b_merged;  // MN-major operand loaded as one box spanning all its atoms
+};
+
+struct TileDesc {
+  Seg seg[4];
+  int nseg;
+  int a_f, b_f;    // fixed coordinate of A / B (row start of K-major, column start of MN-major)
+  int a_c1, b_c1;  // 1: coordinate 1 is the segment's class
+  long long rbase;
+  int rstride, roff;
+  long long rlimit;
+  long long cbase;
+};
+
+// ------------------------------------------------------------------ PTX glue
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long gtime() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok;
+}
+// Bounded wait by one thread.  Returns false if the kernel was aborted or the
+// wait ran out (which records the timeout and aborts the kernel).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const unsigned long long t0 = gtime();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u) {
+      if (*abort) return false;
+      if (gtime() - t0 > kWaitNs) {
+        flag_device_error(kDevTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait used during teardown: never aborts early, gives up after the limit.
+__device__ __noinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = gtime();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 255u) == 255u && gtime() - t0 > kWaitNs) {
+      flag_device_error(kDevTimeout);
+      return;
+    }
+  }
+}
+// The whole warp waits on lane 0's bounded wait (first probe inline).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ok = 0;
+  if (lane == 0) ok = (mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort)) ? 1u : 0u;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+
+__device__ __forceinline__ void tma_load(const CUtensorMap* map, uint32_t dst, uint64_t* bar,
+                                         int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"((unsigned long long)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                          int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          (unsigned long long)map),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- CTA-pair (cta_group::2) helpers
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA ``rank`` of the cluster.
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// TMA load whose completion counts on an mbarrier that may sit in the peer CTA.
+__device__ __forceinline__ void tma_load_pair(const CUtensorMap* map, uint32_t dst, uint32_t bar,
+                                              int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// Arrives on the barrier at this offset in both CTAs of the pair once the
+// pair's previously issued MMAs have completed.
+__device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((unsigned short)3)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load4(const CUtensorMap* map, uint32_t dst, uint64_t* bar,
+                                          int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"((unsigned long long)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load4_pair(const CUtensorMap* map, uint32_t dst, uint32_t bar,
+                                               int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 "version 1").  Field units are
+// 16 bytes.  K-major tiles: rows of 128 B (64 bf16 of K) in 8-row, 1024 B
+// swizzle atoms; SBO = 1024 B between 8-row groups, LBO unused; a K step of 16
+// elements moves the start address by 32 B.  MN-major tiles: per atom, rows of
+// (atom width x 2) B, one row per K index; LBO = distance between atoms along
+// MN, SBO = distance between 8-row K groups.
+__device__ __forceinline__ uint64_t make_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+constexpr uint32_t kLayoutSW128 = 2, kLayoutSW32 = 6;
+
+// Descriptor of an operand tile at shared address ``tile`` (K step 0) and the
+// amount a K step of 16 adds to it (the start-address field is in 16-byte
+// units, so advancing the address is a plain 64-bit add).
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_desc0(uint32_t tile, int aw) {
+  if (!MN) return make_desc(tile, 16, 1024, kLayoutSW128);
+  if (aw == 64) return make_desc(tile, 64 * 128, 1024, kLayoutSW128);
+  return make_desc(tile, 64 * 32, 8 * 32, kLayoutSW32);
+}
+template <bool MN>
+__device__ __forceinline__ uint64_t operand_kstep(int aw) {
+  if (!MN) return 32 >> 4;
+  return aw == 64 ? (16 * 128) >> 4 : (16 * 32) >> 4;
+}
+
+
+// ------------------------------------------------------------- tile layout
+__device__ __forceinline__ void add_seg(TileDesc& d, int k0, int len, int cls, int map) {
+  // merge with the previous segment when the K ranges touch (same class/map)
+  if (d.nseg > 0) {
+    Seg& s = d.seg[d.nseg - 1];
+    if (s.cls == cls && s.map == map && s.k0 + s.len == k0) { s.len += len; return; }
+  }
+  d.seg[d.nseg].k0 = k0;
+  d.seg[d.nseg].len = len;
+  d.seg[d.nseg].cls = cls;
+  d.seg[d.nseg].map = map;
+  ++d.nseg;
+}
+
+// The p1 that makes pair (p0, p1) diagonal: the row type of class p0 for the
+// row-typed ops, p0 itself for the square product and dW.
+__device__ __forceinline__ int type_of_class(const Params& p, int c) {
+  const int t = c + p.off;  // c, off < q
+  return t >= p.q ? t - p.q : t;
+}
+__device__ __forceinline__ int diag_partner(const Params& p, int p0) {
+  return (p.op == OP_SQUARE || p.op == OP_DW) ? p0 : type_of_class(p, p0);
+}
+
+__device__ __forceinline__ void pair_of(const Params& p, int pr, int& p0, int& p1) {
+  if (p.npairs_list) {
+    const int v = p.pairs[pr];
+    p0 = v >> 8;
+    p1 = v & 255;
+    return;
+  }
+  const int q = p.q, nd = q * (q - 1);
+  int r = pr;
+  if (p.diag_first) {
+    if (r < q) { p0 = r; p1 = diag_partner(p, r); return; }
+    r -= q;
+  } else if (r >= nd) {
+    p0 = r - nd;
+    p1 = diag_partner(p, p0);
+    return;
+  }
+  p0 = (int)fdiv((uint32_t)r, p.div_qm1);
+  const int j = r - p0 * (q - 1), dg = diag_partner(p, p0);
+  p1 = j < dg ? j : j + 1;
+}
+
+// tile = (pair_rank * n1 + i1) * n3 + i3; the pair is (i0, i2) of the op.
+__device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
+  const int t3 = (int)fdiv((uint32_t)tile, p.div_n3);
+  const int i3 = tile - t3 * p.n3;
+  const int pr = (int)fdiv((uint32_t)t3, p.div_n1);
+  const int i1 = t3 - pr * p.n1;
+  int i0, i2;
+  pair_of(p, pr, i0, i2);
+  d.nseg = 0;
+  d.rstride = 1;
+  d.roff = 0;
+  d.rlimit = LLONG_MAX;
+  switch (p.op) {
+    case OP_FWD:
+    case OP_SWIGLU: {  // i0 class, i1 token block, i2 output group k, i3 column block
+      const int c = i0, k = i2, t = type_of_class(p, c);
+      int mem[4];
+      const int n = table_members(p.law, p.q, t, k, mem);
+      for (int s = 0; s < n; ++s) add_seg(d, mem[s] * p.bi, p.bi, c, 0);
+      const int xrow0 = i1 * p.xr, wcol0 = k * p.bo + i3 * p.wn;
+      if (!p.swap) { d.a_f = xrow0; d.a_c1 = 1; d.b_f = wcol0; d.b_c1 = 0; }
+      else { d.a_f = wcol0; d.a_c1 = 0; d.b_f = xrow0; d.b_c1 = 1; }
+      d.rbase = xrow0; d.rstride = p.qv; d.roff = c; d.rlimit = p.Mq; d.cbase = wcol0;
+      break;
+    }
+    case OP_SQUARE: {  // i0 row block i, i1 128-row slab, i2 column block k, i3 column slab
+      const int i = i0, k = i2;
+      int mem[4];
+      const int n = table_members(p.law, p.q, i, k, mem);
+      for (int s = 0; s < n; ++s) add_seg(d, mem[s] * p.bi, p.bi, 0, 0);
+      d.a_f = i * p.bi + i1 * 128; d.a_c1 = 0;
+      d.b_f = k * p.bo + i3 * p.wn; d.b_c1 = 0;
+      d.rbase = d.a_f; d.cbase = d.b_f;
+      break;
+    }
+    case OP_DX: {  // i0 class, i1 token block, i2 input group a, i3 column block of group a
+      const int c = i0, a = i2, t = type_of_class(p, c);
+      for (int k = 0; k < p.q; ++k)
+        if (in_table(p.law, t, k, a)) add_seg(d, k * p.bo, p.bo, c, 0);
+      d.a_f = i1 * 128; d.a_c1 = 1;
+      d.b_f = a * p.bi + i3 * p.wn; d.b_c1 = 0;
+      d.rbase = i1 * 128; d.rstride = p.qv; d.roff = c; d.rlimit = p.Mq;
+      d.cbase = d.b_f;
+      break;
+    }
+    case OP_DW: {  // i0 group a, i2 group k; (i1, i3) = (row slab, column block) or swapped
+      const int a = i0, k = i2;
+      const int mb = p.swap ? i3 : i1, nb = p.swap ? i1 : i3;
+      if (p.law == AAL_LAW_Q && a == k) {
+        add_seg(d, 0, (int)p.Mall, 0, 1);  // every type uses the diagonal block
+      } else {
+        for (int c = 0; c < p.qv; ++c)
+          if (in_table(p.law, type_of_class(p, c), k, a)) add_seg(d, 0, (int)p.Mq, c, 0);
+      }
+      const int xf = a * p.bi + (p.swap ? nb * p.wn : mb * 128);
+      const int yf = k * p.bo + (p.swap ? mb * 128 : nb * p.wn);
+      if (!p.swap) { d.a_f = xf; d.b_f = yf; } else { d.a_f = yf; d.b_f = xf; }
+      d.a_c1 = 1; d.b_c1 = 1;
+      d.rbase = xf; d.cbase = yf;
+      break;
+    }
+  }
+}
+
+__device__ __forceinline__ int seg_chunks(const Seg& s) { return (s.len + 63) >> 6; }
+
+// --------------------------------------------------------------- the kernel
+// A_MN / B_MN: operand tiles stored MN-major (else K-major).
+// DUAL: 0 one MMA per K step; 1 two B operands (gate/up); 2 two A operands.
+// PAIR: the tile is computed by a CTA pair with tcgen05 cta_group::2 (M = 256);
+// each CTA loads its half of A's rows and of B's columns (for DUAL == 1, CTA r
+// loads B operand r), only the pair's first CTA issues MMAs and counts the
+// transaction bytes, and each CTA drains its own 128 TMEM lanes.
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR>
+__global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t done_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t smem0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const int S = p.stages;
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool issuer = !PAIR || rank == 0;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * kEpiWarps);
+    }
+    mbar_init(&done_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    if (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&s_tmem)),
+                   "r"(p.tmem_cols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&s_tmem)),
+                   "r"(p.tmem_cols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    uint32_t it = 0, st = 0, ph = 0;
+    bool ok = true;
+    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep) {
+      TileDesc d;
+      describe(p, tile, d);
+      for (int s = 0; s < d.nseg && ok; ++s) {
+        const Seg sg = d.seg[s];
+        const int nch = seg_chunks(sg);
+        for (int kc = 0; kc < nch; ++kc) {
+          if (!warp_wait(&empty_bar[st], ph ^ 1u, &s_abort)) { ok = false; break; }
+          {
+            // The boxes of a stage are issued by separate lanes: one thread
+            // issuing them back to back serialises the TMA requests.
+            const uint32_t base = smem0 + st * p.stage_bytes;
+            const int kofs = sg.k0 + kc * 64;
+            const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
+            if (lane == 0 && issuer) mbar_expect_tx(&full_bar[st], (PAIR ? 2u : 1u) * p.stage_bytes);
+            const int na = DUAL == 2 ? 2 : 1;
+            const int nb = (DUAL == 1 && !PAIR) ? 2 : 1;
+            const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
+            const int nB = (B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1;  // boxes per B operand
+            const int arow = PAIR ? (int)rank * 128 : 0;  // this CTA's half of the A tile
+            const int bsh = (PAIR && DUAL != 1) ? (int)rank * p.b_rows : 0;
+            for (int bx = lane; bx < na * nA + nb * nB; bx += 32) {
+              if (bx < na * nA) {
+                const int o = bx / nA, at = bx - o * nA;
+                const CUtensorMap* m = &p.mapA[DUAL == 2 ? o : sg.map];
+                const int c1 = d.a_c1 ? sg.cls : 0;
+                const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
+                if (A_MN && p.a_merged) {
+                  // all atoms at once: coordinates (col in atom, class, K row, atom)
+                  const int x3 = (d.a_f + arow) / p.a_aw;
+                  if (PAIR) tma_load4_pair(m, dst, fb, 0, c1, kofs, x3);
+                  else tma_load4(m, dst, &full_bar[st], 0, c1, kofs, x3);
+                } else {
+                  const int x0 = A_MN ? d.a_f + arow + at * p.a_aw : kofs;
+                  const int x2 = A_MN ? kofs : d.a_f + arow;
+                  if (PAIR) tma_load_pair(m, dst, fb, x0, c1, x2);
+                  else tma_load(m, dst, &full_bar[st], x0, c1, x2);
+                }
+              } else {
+                // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
+                // the MMA's B, or, with two B operands, all of operand r
+                const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : sg.map;
+                const CUtensorMap* m = &p.mapB[mop];
+                const int c1 = d.b_c1 ? sg.cls : 0;
+                const uint32_t dst =
+                    base + na * p.a_bytes + o * p.b_bytes + (B_MN ? at * (p.b_aw * 2 * 64) : 0);
+                if (B_MN && p.b_merged) {
+                  const int x3 = (d.b_f + bsh) / p.b_aw;
+                  if (PAIR) tma_load4_pair(m, dst, fb, 0, c1, kofs, x3);
+                  else tma_load4(m, dst, &full_bar[st], 0, c1, kofs, x3);
+                } else {
+                  const int x0 = B_MN ? d.b_f + bsh + at * p.b_aw : kofs;
+                  const int x2 = B_MN ? kofs : d.b_f + bsh;
+                  if (PAIR) tma_load_pair(m, dst, fb, x0, c1, x2);
+                  else tma_load(m, dst, &full_bar[st], x0, c1, x2);
+                }
+              }
+            }
+          }
+          __syncwarp();
+          ++it;
+          if (++st == (uint32_t)S) { st = 0; ph ^= 1u; }
+        }
+      }
+    }
+    // let every copy this CTA issued land before the CTA can exit (for a pair
+    // the pair's first CTA sees both halves on its own barriers)
+    if (lane == 0 && issuer) {
+      for (int st = 0; st < S; ++st) {
+        if ((uint32_t)st >= it) break;
+        const uint32_t last = st + ((it - 1 - st) / S) * S;
+        mbar_wait_teardown(&full_bar[st], (last / S) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (issuer && lane == 0) {
+      // One thread issues; a running stage index and phase bit replace
+      // divisions, so the next MMAs follow the previous ones closely.
+      uint32_t st = 0, ph = 0, tl = 0;
+      bool ok = true;
+      const int na = DUAL == 2 ? 2 : 1;
+      // Descriptors of stage 0 and their per-stage and per-K-step increments,
+      // built once: the issue loop below only adds.
+      const uint64_t dA0 = operand_desc0<A_MN>(smem0, p.a_aw);
+      const uint64_t dA1 = operand_desc0<A_MN>(smem0 + p.a_bytes, p.a_aw);
+      const uint64_t dB0 = operand_desc0<B_MN>(smem0 + na * p.a_bytes, p.b_aw);
+      const uint64_t dB1 = operand_desc0<B_MN>(smem0 + na * p.a_bytes + p.b_bytes, p.b_aw);
+      const uint64_t dstage = p.stage_bytes >> 4;
+      const uint64_t kA = operand_kstep<A_MN>(p.a_aw), kB = operand_kstep<B_MN>(p.b_aw);
+      const uint32_t idesc = (PAIR ? (DUAL == 1 ? p.idesc2 : p.idesc)
+                                   : ((DUAL == 1 && p.fuse_b) ? p.idesc2 : p.idesc));
+      const bool single = PAIR || DUAL == 0 || (DUAL == 1 && p.fuse_b);
+      uint64_t so = 0;  // dstage * st
+      for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++tl) {
+        TileDesc d;
+        describe(p, tile, d);
+        const uint32_t buf = tl & 1u, use = tl >> 1;
+        if (!(mbar_try_wait(&tempty_bar[buf], (use & 1u) ^ 1u) ||
+              mbar_wait(&tempty_bar[buf], (use & 1u) ^ 1u, &s_abort))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t acc0 = tmem + buf * p.acc_cols;
+        const uint32_t acc1 = acc0 + p.n_mma;
+        uint32_t accumulate = 0;
+        for (int s = 0; s < d.nseg && ok; ++s) {
+          const int len = d.seg[s].len;
+          for (int rem = len; rem > 0; rem -= 64) {
+            if (!(mbar_try_wait(&full_bar[st], ph) || mbar_wait(&full_bar[st], ph, &s_abort))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t a0 = dA0 + so, b0 = dB0 + so;
+            const uint64_t a1 = dA1 + so, b1 = dB1 + so;
+            if (rem >= 64) {
+              // the common full chunk: four K steps, unrolled
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                if (PAIR) {
+                  tc_mma_pair(acc0, a0 + ks * kA, b0 + ks * kB, idesc, accumulate);
+                } else if (single) {
+                  tc_mma(acc0, a0 + ks * kA, b0 + ks * kB, idesc, accumulate);
+                } else {
+                  tc_mma(acc0, a0 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
+                  if (DUAL == 1) tc_mma(acc1, a0 + ks * kA, b1 + ks * kB, p.idesc, accumulate);
+                  if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
+                }
+                accumulate = 1;
+              }
+            } else {
+              const int ksteps = (rem + 15) >> 4;
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const uint64_t da = a0 + ks * kA, db = b0 + ks * kB;
+                if (PAIR) {
+                  tc_mma_pair(acc0, da, db, idesc, accumulate);
+                } else if (single) {
+                  tc_mma(acc0, da, db, idesc, accumulate);
+                } else {
+                  tc_mma(acc0, da, db, p.idesc, accumulate);
+                  if (DUAL == 1) tc_mma(acc1, da, b1 + ks * kB, p.idesc, accumulate);
+                  if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, db, p.idesc, accumulate);
+                }
+                accumulate = 1;
+              }
+            }
+            // frees the stage (in both CTAs of a pair) once these MMAs have read it
+            if (PAIR) tc_commit_pair_mc(&empty_bar[st]);
+            else tc_commit(&empty_bar[st]);
+            if (++st == (uint32_t)S) { st = 0; ph ^= 1u; so = 0; }
+            else so += dstage;
+          }
+        }
+        if (!ok) break;
+        if (PAIR) tc_commit_pair_mc(&tfull_bar[buf]);
+        else tc_commit(&tfull_bar[buf]);
+      }
+      // wait for every MMA this CTA issued before TMEM is released
+      if (PAIR) tc_commit_pair_mc(&done_bar);
+      else tc_commit(&done_bar);
+      mbar_wait_teardown(&done_bar, 0);
+    }
+  } else {
+    // ------------------------------------------------------ epilogue
+    const int quarter = warp & 3;             // TMEM lanes this warp may read
+    const int half = (warp - 2) / 4;          // which of the 16-column chunks it drains
+    const int row_in_tile = quarter * 32 + lane;
+    // two 1 KB staging buffers per epilogue warp, after the pipeline stages
+    const uint32_t stage_buf = smem0 + S * p.stage_bytes + (warp - 2) * 2048;
+    uint32_t nstore = 0;
+    uint32_t tl = 0;
+    const int erow = PAIR ? (int)rank * 128 : 0;  // this CTA's 128 rows of the pair's tile
+    for (int tile = tile0; tile < p.ntiles; tile += tstep, ++tl) {
+      TileDesc d;
+      describe(p, tile, d);
+      d.rbase += erow;
+      const uint32_t buf = tl & 1u, use = tl >> 1;
+      if (!warp_wait(&tfull_bar[buf], use & 1u, &s_abort)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * p.acc_cols;
+      const uint32_t tempty_addr =
+          PAIR ? mapa_rank(smem_u32(&tempty_bar[buf]), 0) : smem_u32(&tempty_bar[buf]);
+      const int nch = (p.n_mma / 16 + 1 - half) / 2;  // chunks c0 = half*16 + 32*i
+      for (int ci = 0; ci < nch; ++ci) {
+        const int c0 = half * 16 + 32 * ci;
+        float v[16];
+        tmem_ld16(tbase + c0, v);
+        if (p.swiglu) {
+          float u[16];
+          tmem_ld16(tbase + p.n_mma + c0, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            // silu(g) * u with g * sigmoid(g); large negative g gives 0
+            const float sg = __frcp_rn(1.0f + __expf(-v[j]));
+            v[j] = v[j] * sg * u[j];
+          }
+        } else {
+          tmem_wait_ld();
+        }
+        if (ci == nch - 1) {
+          // the accumulator is in registers: hand the TMEM buffer back early
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (PAIR) mbar_arrive_remote(tempty_addr);
+            else mbar_arrive(&tempty_bar[buf]);
+          }
+        }
+        if (p.tma_store) {
+          const uint32_t sb = stage_buf + (nstore & 1u) * 1024;
+          if (nstore >= 2) {
+            if (lane == 0) bulk_wait_read1();  // the buffer's previous store has read it
+            __syncwarp();
+          }
+          if (!p.swap) {
+            // 32 rows x 16 columns, 32-byte rows, 32-byte swizzle
+            uint4 w[2];
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            const uint32_t row = sb + lane * 32;
+            const uint32_t flip = (lane >> 2) & 1u;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((0u ^ flip) << 4)),
+                         "r"(w[0].x), "r"(w[0].y), "r"(w[0].z), "r"(w[0].w));
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((1u ^ flip) << 4)),
+                         "r"(w[1].x), "r"(w[1].y), "r"(w[1].z), "r"(w[1].w));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store(&p.mapOut, sb, (int)(d.cbase + c0), d.roff,
+                        (int)(d.rbase + quarter * 32));
+              bulk_commit();
+            }
+          } else {
+            // 16 rows x 32 columns (this warp's 32 TMEM lanes), 64-byte rows
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(sb + j * 64 + lane * 2),
+                           "h"(*reinterpret_cast<const unsigned short*>(&hv)));
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store(&p.mapOut, sb, (int)(d.cbase + quarter * 32), d.roff,
+                        (int)(d.rbase + c0));
+              bulk_commit();
+            }
+          }
+          ++nstore;
+        } else if (!p.swap) {
+          const long long x = d.rbase + row_in_tile;
+          if (x < d.rlimit) {
+            __nv_bfloat16* dst = p.out + (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
+            if (p.accumulate) {
+              uint4 o0 = reinterpret_cast<const uint4*>(dst)[0];
+              uint4 o1 = reinterpret_cast<const uint4*>(dst)[1];
+              const __nv_bfloat16* ob0 = reinterpret_cast<const __nv_bfloat16*>(&o0);
+              const __nv_bfloat16* ob1 = reinterpret_cast<const __nv_bfloat16*>(&o1);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                v[j] += __bfloat162float(ob0[j]);
+                v[8 + j] += __bfloat162float(ob1[j]);
+              }
+            }
+            uint4 w[2];
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            reinterpret_cast<uint4*>(dst)[0] = w[0];
+            reinterpret_cast<uint4*>(dst)[1] = w[1];
+          }
+        } else {
+          const long long col = d.cbase + row_in_tile;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const long long x = d.rbase + c0 + j;
+            if (x < d.rlimit) {
+              __nv_bfloat16* dst = p.out + (x * d.rstride + d.roff) * p.ldo + col;
+              float val = v[j];
+              if (p.accumulate) val += __bfloat162float(*dst);
+              *dst = __float2bfloat16_rn(val);
+            }
+          }
+        }
+      }
+      if (nch == 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_remote(tempty_addr);
+          else mbar_arrive(&tempty_bar[buf]);
+        }
+      }
+    }
+    // every TMA store of this warp must have finished before the CTA exits
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // a pair stays resident until the peer is done with its shared memory and TMEM
+  if (PAIR) cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(p.tmem_cols));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(p.tmem_cols));
+  }
+}
+
+// ------------------------------------------------------------ host planning
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// A row-major bf16 matrix [rows, cols] (leading dimension ld) seen as
+// [rows/qv][qv][cols]; box {box0 elements, 1, box2 rows}.
+static bool make_map(CUtensorMap* m, const void* ptr, long long rows, long long cols, long long ld,
+                     int qv, int box0, int box2, int swizzle_bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rows % qv) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)qv, (cuuint64_t)(rows / qv)};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld * 2), (cuuint64_t)(ld * 2 * qv)};
+  cuuint32_t box[3] = {(cuuint32_t)box0, 1u, (cuuint32_t)box2};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                          : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// K-major operand tile: box {64 K elements, 1, rows}.
+static bool map_kmajor(CUtensorMap* m, const aal_mat& t, int qv, int rows_box) {
+  return make_map(m, t.ptr, t.rows, t.cols, t.ld, qv, 64, rows_box, 128);
+}
+// MN-major operand tile: box {atom width, 1, 64 K rows}.
+static bool map_mnmajor(CUtensorMap* m, const aal_mat& t, int qv, int aw) {
+  return make_map(m, t.ptr, t.rows, t.cols, t.ld, qv, aw, 64, aw == 64 ? 128 : 32);
+}
+// MN-major operand tile in one box: the matrix seen as
+// [cols/aw][rows/qv][qv][aw] (atom index outermost), box {aw, 1, 64, natoms};
+// shared memory then holds the atoms one after another, as the MMA reads them.
+static bool map_mnmajor_merged(CUtensorMap* m, const aal_mat& t, int qv, int aw, int natoms) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || t.rows % qv || t.cols % aw || natoms < 1 || natoms > 256) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)aw, (cuuint64_t)qv, (cuuint64_t)(t.rows / qv),
+                        (cuuint64_t)(t.cols / aw)};
+  cuuint64_t strides[3] = {(cuuint64_t)(t.ld * 2), (cuuint64_t)(t.ld * 2 * qv),
+                           (cuuint64_t)(aw * 2)};
+  cuuint32_t box[4] = {(cuuint32_t)aw, 1u, 64u, (cuuint32_t)natoms};
+  cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  const CUresult r =
+      enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(t.ptr), dims, strides, box, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, aw == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+// Builds the one-box map when the encoder accepts it, else the per-atom map.
+static bool map_mn(CUtensorMap* m, const aal_mat& t, int qv, int aw, int extent, int* merged) {
+  if (map_mnmajor_merged(m, t, qv, aw, extent / aw)) { *merged = 1; return true; }
+  *merged = 0;
+  return map_mnmajor(m, t, qv, aw);
+}
+
+// Output map for the TMA-store epilogue: 32 rows x 16 columns per store
+// (32-byte swizzle), or 16 rows x 32 columns when TMEM lanes are columns.
+static bool out_map(Params& p, const aal_mat& out, int qv) {
+  p.tma_store = p.accumulate ? 0 : 1;
+  if (!p.tma_store) return true;
+  if (p.swap) return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 32, 16, 0);
+  return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 16, 32, 32);
+}
+
+static bool tc_aligned(const aal_mat& m) {
+  return m.dtype == AAL_BF16 && ((uintptr_t)m.ptr % 16) == 0 && (m.ld % 8) == 0;
+}
+
+// Largest N <= cap with ext % N == 0 and N % 16 == 0, preferring multiples of 64.
+static int pick_n(long long ext, int cap) {
+  int best = 0;
+  for (int n = cap; n >= 16; n -= 16) {
+    if (ext % n) continue;
+    if (n % 64 == 0) return n;
+    if (!best) best = n;
+  }
+  return best;
+}
+
+static uint32_t make_idesc(int m, int n, bool a_mn, bool b_mn) {
+  uint32_t d = 0;
+  d |= 1u << 4;   // D format: f32
+  d |= 1u << 7;   // A format: bf16
+  d |= 1u << 10;  // B format: bf16
+  d |= (a_mn ? 1u : 0u) << 15;
+  d |= (b_mn ? 1u : 0u) << 16;
+  d |= (uint32_t)(n >> 3) << 17;
+  d |= (uint32_t)(m >> 4) << 24;
+  return d;
+}
+
+static int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+static bool is_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  return major == 10;
+}
+
+// Fills the pipeline sizes and TMEM allocation; false if they do not fit.
+static bool finish_plan(Params& p, int dual, bool pair = false) {
+  const int na = dual == 2 ? 2 : 1, nb = (dual == 1 && !pair) ? 2 : 1;
+  p.a_bytes = (uint32_t)p.a_rows * 128u;
+  p.b_bytes = (uint32_t)p.b_rows * 128u;
+  p.stage_bytes = na * p.a_bytes + nb * p.b_bytes;
+  p.stages = (kSmemBudget - kEpiSmem) / (int)p.stage_bytes;
+  if (p.stages > kMaxStages) p.stages = kMaxStages;
+  if (p.stages < 2) return false;
+  p.acc_cols = p.n_mma * (dual ? 2 : 1);
+  const int need = 2 * p.acc_cols;
+  if (need > 512) return false;
+  uint32_t cols = 32;
+  while ((int)cols < need) cols <<= 1;
+  p.tmem_cols = cols;
+  p.ntiles = 0;
+  return true;
+}
+
+// Block products behind the tile pair (p0, p1) of the op: the table-entry size
+// for the forward ops, the number of k (dX) or classes (dW) that use a block.
+static int pair_cost(const Params& p, int p0, int p1) {
+  int mem[4];
+  switch (p.op) {
+    case OP_FWD:
+    case OP_SWIGLU: return table_members(p.law, p.q, (p0 + p.off) % p.q, p1, mem);
+    case OP_SQUARE: return table_members(p.law, p.q, p0, p1, mem);
+    case OP_DX: {
+      int n = 0;
+      for (int k = 0; k < p.q; ++k) n += in_table(p.law, (p0 + p.off) % p.q, k, p1) ? 1 : 0;
+      return n;
+    }
+    default: {
+      if (p.law == AAL_LAW_Q && p0 == p1) return p.q;
+      int n = 0;
+      for (int c = 0; c < p.qv; ++c) n += in_table(p.law, (c + p.off) % p.q, p1, p0) ? 1 : 0;
+      return n;
+    }
+  }
+}
+
+// Orders the q*q tile pairs longest first.
+static void order_pairs(Params& p) {
+  const int q = p.q;
+  if (q * q <= kMaxPairs && q <= 256) {
+    int n = 0;
+    for (int cost = 4 * q; cost >= 0; --cost)
+      for (int p0 = 0; p0 < q; ++p0)
+        for (int p1 = 0; p1 < q; ++p1)
+          if (pair_cost(p, p0, p1) == cost) p.pairs[n++] = (uint16_t)(p0 << 8 | p1);
+    p.npairs_list = n;
+  } else {
+    p.npairs_list = 0;
+    p.diag_first = (p.op == OP_DX || p.op == OP_DW) ? 1 : 0;
+  }
+}
+
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false>
+static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
+  if (ntiles <= 0) return AAL_OK;
+  if (ntiles > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  p.ntiles = (int)ntiles;
+  order_pairs(p);
+  p.div_n1 = make_fastdiv((uint32_t)p.n1);
+  p.div_n3 = make_fastdiv((uint32_t)p.n3);
+  p.div_qm1 = make_fastdiv((uint32_t)(p.q > 1 ? p.q - 1 : 1));
+  const size_t smem = (size_t)p.stages * p.stage_bytes + kEpiSmem + 1024;
+  static unsigned long long attr_set = 0;  // one bit per device ordinal
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return AAL_ERR_CUDA;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    if (cudaFuncSetAttribute(k_tc<A_MN, B_MN, DUAL, PAIR>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBudget + 1024) != cudaSuccess)
+      return AAL_ERR_CUDA;
+    attr_set |= bit;
+  }
+  const int sms = num_sms();
+  if (!PAIR) {
+    const int grid = (int)(ntiles < sms ? ntiles : sms);
+    k_tc<A_MN, B_MN, DUAL, false><<<grid, kThreads, smem, s>>>(p);
+    note_launch();
+    return cuda_status(cudaGetLastError());
+  }
+  const int pairs = (int)(ntiles < sms / 2 ? ntiles : sms / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, true>, p);
+  note_launch();
+  return cuda_status(e);
+}
+
+// AAL_TC_PAIR=0 in the environment turns the CTA-pair mode off.
+static bool pair_disabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_TC_PAIR");
+    v = (e && e[0] == '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+static bool position_rule_ok(const RowTypes& rt, int q, long long rows) {
+  return rt.kind == kTypesPosition && rt.seq_len % q == 0 && rows % q == 0 && rows > 0;
+}
+
+static void base_params(Params& p, int law, int q, const RowTypes& rt, long long rows) {
+  memset(&p, 0, sizeof(p));
+  p.law = law;
+  p.q = q;
+  p.off = (int)(rt.pos_offset % q);
+  p.qv = q;
+  p.Mq = rows / q;
+  p.Mall = rows;
+}
+
+}  // namespace tc
+
+using namespace tc;
+
+// Projection and fused gate/up share the planning; ``Wu`` null -> projection.
+static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long rows,
+                                  const aal_mat& X, const aal_mat& Wg, const aal_mat* Wu,
+                                  const aal_mat& Y, cudaStream_t s) {
+  if (!is_sm100() || !position_rule_ok(rt, q, rows)) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(X) || !tc_aligned(Wg) || !tc_aligned(Y) || (Wu && !tc_aligned(*Wu)))
+    return AAL_ERR_UNSUPPORTED;
+  const long long bi = X.cols / q, bo = Wg.cols / q;
+  if (bi % 16 || bo % 16 || bi > INT_MAX || bo > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  const bool dual = Wu != nullptr;
+  Params p;
+  base_params(p, law, q, rt, rows);
+  p.op = dual ? OP_SWIGLU : OP_FWD;
+  p.bi = (int)bi;
+  p.bo = (int)bo;
+  p.swiglu = dual;
+  p.out = (__nv_bfloat16*)Y.ptr;
+  p.ldo = Y.ld;
+  const bool swap = p.Mq < 128 && bo % 128 == 0;
+  long long ntiles;
+  // CTA pair (M = 256): enough rows per class, and each CTA's half of B a
+  // whole number of 16-column atoms
+  const int npair = pick_n(bo, dual ? 128 : 256);
+  const bool pair = !swap && p.Mq >= 256 && npair && (dual ? npair == 128 : (npair / 2) % 16 == 0) &&
+                    !pair_disabled();
+  if (pair) {
+    const int n = npair;
+    p.swap = 0;
+    p.xr = 256;
+    p.wn = n;
+    p.n_mma = n;  // per-operand width; the MMA spans 2n with two operands
+    p.a_rows = 128;
+    p.b_rows = dual ? n : n / 2;
+    p.b_aw = p.b_rows % 64 == 0 ? 64 : 16;
+    p.fuse_b = dual;
+    p.idesc = make_idesc(256, n, false, true);
+    p.idesc2 = dual ? make_idesc(256, 2 * n, false, true) : 0;
+    if (!finish_plan(p, dual ? 1 : 0, true)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], X, q, 128)) return AAL_ERR_UNSUPPORTED;
+    int mg1 = 1;
+    if (!map_mn(&p.mapB[0], Wg, 1, p.b_aw, p.b_rows, &p.b_merged)) return AAL_ERR_UNSUPPORTED;
+    if (dual && !map_mn(&p.mapB[1], *Wu, 1, p.b_aw, p.b_rows, &mg1)) return AAL_ERR_UNSUPPORTED;
+    if (!mg1 && p.b_merged) {  // both operands must use the same form
+      p.b_merged = 0;
+      if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    }
+    if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = (int)((p.Mq + 255) / 256);
+    p.n2 = q;
+    p.n3 = (int)(bo / n);
+    ntiles = (long long)q * p.n1 * p.n2 * p.n3;
+    return dual ? launch<false, true, 1, true>(p, ntiles, s) : launch<false, true, 0, true>(p, ntiles, s);
+  }
+  if (!swap) {
+    const int n = pick_n(bo, dual ? 128 : 256);
+    if (!n) return AAL_ERR_UNSUPPORTED;
+    p.swap = 0;
+    p.xr = 128;
+    p.wn = n;
+    p.n_mma = n;
+    p.a_rows = 128;
+    p.b_rows = n;
+    p.b_aw = n % 64 == 0 ? 64 : 16;
+    p.idesc = make_idesc(128, n, false, true);
+    // gate and up tiles form one MN-major operand when the atom stride is uniform
+    p.fuse_b = dual && p.b_aw == 64 && 2 * n <= 256;
+    p.idesc2 = p.fuse_b ? make_idesc(128, 2 * n, false, true) : 0;
+    if (!finish_plan(p, dual ? 1 : 0)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], X, q, 128)) return AAL_ERR_UNSUPPORTED;
+    int mg1 = 1;
+    if (!map_mn(&p.mapB[0], Wg, 1, p.b_aw, p.b_rows, &p.b_merged)) return AAL_ERR_UNSUPPORTED;
+    if (dual && !map_mn(&p.mapB[1], *Wu, 1, p.b_aw, p.b_rows, &mg1)) return AAL_ERR_UNSUPPORTED;
+    if (!mg1 && p.b_merged) {
+      p.b_merged = 0;
+      if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    }
+    if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = (int)((p.Mq + 127) / 128);
+    p.n2 = q;
+    p.n3 = (int)(bo / n);
+    ntiles = (long long)q * p.n1 * p.n2 * p.n3;
+    return dual ? launch<false, true, 1>(p, ntiles, s) : launch<false, true, 0>(p, ntiles, s);
+  }
+  const int ntok = (int)((p.Mq + 15) / 16 * 16);
+  p.swap = 1;
+  p.xr = ntok;
+  p.wn = 128;
+  p.n_mma = ntok;
+  p.a_rows = 128;
+  p.b_rows = ntok;
+  p.a_aw = 64;
+  p.idesc = make_idesc(128, ntok, true, false);
+  if (!finish_plan(p, dual ? 2 : 0)) return AAL_ERR_UNSUPPORTED;
+  int mg1 = 1;
+  if (!map_mn(&p.mapA[0], Wg, 1, 64, 128, &p.a_merged)) return AAL_ERR_UNSUPPORTED;
+  if (dual && !map_mn(&p.mapA[1], *Wu, 1, 64, 128, &mg1)) return AAL_ERR_UNSUPPORTED;
+  if (!mg1 && p.a_merged) {
+    p.a_merged = 0;
+    if (!map_mnmajor(&p.mapA[0], Wg, 1, 64)) return AAL_ERR_UNSUPPORTED;
+  }
+  if (!map_kmajor(&p.mapB[0], X, q, ntok)) return AAL_ERR_UNSUPPORTED;
+  if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+  p.n1 = 1;
+  p.n2 = q;
+  p.n3 = (int)(bo / 128);
+  ntiles = (long long)q * p.n2 * p.n3;
+  return dual ? launch<true, false, 2>(p, ntiles, s) : launch<true, false, 0>(p, ntiles, s);
+}
+
+aal_status tc_project(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                      const aal_mat& W, const aal_mat& Y, cudaStream_t s) {
+  return tc_project_impl(law, q, rt, rows, X, W, nullptr, Y, s);
+}
+
+aal_status tc_swiglu_gate_up(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                             const aal_mat& Wg, const aal_mat& Wu, const aal_mat& H,
+                             cudaStream_t s) {
+  return tc_project_impl(law, q, rt, rows, X, Wg, &Wu, H, s);
+}
+
+aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
+                             const aal_mat& W, const aal_mat& dX, cudaStream_t s) {
+  if (!is_sm100() || !position_rule_ok(rt, q, rows)) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(dY) || !tc_aligned(W) || !tc_aligned(dX)) return AAL_ERR_UNSUPPORTED;
+  const long long bi = W.rows / q, bo = W.cols / q;
+  if (bi % 16 || bo % 16) return AAL_ERR_UNSUPPORTED;
+  Params p;
+  base_params(p, law, q, rt, rows);
+  p.op = OP_DX;
+  p.bi = (int)bi;
+  p.bo = (int)bo;
+  p.out = (__nv_bfloat16*)dX.ptr;
+  p.ldo = dX.ld;
+  const int n = pick_n(bi, 256);
+  if (!n) return AAL_ERR_UNSUPPORTED;
+  p.xr = 128;
+  p.wn = n;
+  p.n_mma = n;
+  p.a_rows = 128;
+  p.b_rows = n;
+  p.idesc = make_idesc(128, n, false, false);
+  if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapA[0], dY, q, 128)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapB[0], W, 1, n)) return AAL_ERR_UNSUPPORTED;
+  if (!out_map(p, dX, q)) return AAL_ERR_UNSUPPORTED;
+  p.n1 = (int)((p.Mq + 127) / 128);
+  p.n2 = q;
+  p.n3 = (int)(bi / n);
+  return launch<false, false, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+}
+
+aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
+                             const aal_mat& dY, const aal_mat& dW, int accumulate,
+                             cudaStream_t s) {
+  if (!is_sm100() || !position_rule_ok(rt, q, rows)) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(X) || !tc_aligned(dY) || !tc_aligned(dW)) return AAL_ERR_UNSUPPORTED;
+  const long long bi = dW.rows / q, bo = dW.cols / q;
+  if (bi % 16 || bo % 16 || rows > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  Params p;
+  base_params(p, law, q, rt, rows);
+  p.op = OP_DW;
+  p.bi = (int)bi;
+  p.bo = (int)bo;
+  p.out = (__nv_bfloat16*)dW.ptr;
+  p.ldo = dW.ld;
+  p.accumulate = accumulate ? 1 : 0;
+  // MMA M = 128 features of group a (or of group k when swapped), N the other side
+  const bool swap = bi % 128 != 0;
+  if (swap && bo % 128 != 0) return AAL_ERR_UNSUPPORTED;
+  const int n = pick_n(swap ? bi : bo, 256);
+  if (!n) return AAL_ERR_UNSUPPORTED;
+  p.swap = swap;
+  p.wn = n;
+  p.n_mma = n;
+  p.a_rows = 128;
+  p.b_rows = n;
+  p.a_aw = 64;
+  p.b_aw = n % 64 == 0 ? 64 : 16;
+  p.idesc = make_idesc(128, n, true, true);
+  if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+  const aal_mat& A = swap ? dY : X;
+  const aal_mat& B = swap ? X : dY;
+  {
+    int ma0 = 0, ma1 = 0, mb0 = 0, mb1 = 0;
+    if (!map_mn(&p.mapA[0], A, q, 64, 128, &ma0) || !map_mn(&p.mapA[1], A, 1, 64, 128, &ma1))
+      return AAL_ERR_UNSUPPORTED;
+    if (!map_mn(&p.mapB[0], B, q, p.b_aw, n, &mb0) || !map_mn(&p.mapB[1], B, 1, p.b_aw, n, &mb1))
+      return AAL_ERR_UNSUPPORTED;
+    if (!(ma0 && ma1)) {
+      if (!map_mnmajor(&p.mapA[0], A, q, 64) || !map_mnmajor(&p.mapA[1], A, 1, 64))
+        return AAL_ERR_UNSUPPORTED;
+    }
+    if (!(mb0 && mb1)) {
+      if (!map_mnmajor(&p.mapB[0], B, q, p.b_aw) || !map_mnmajor(&p.mapB[1], B, 1, p.b_aw))
+        return AAL_ERR_UNSUPPORTED;
+    }
+    p.a_merged = ma0 && ma1;
+    p.b_merged = mb0 && mb1;
+  }
+  if (!out_map(p, dW, 1)) return AAL_ERR_UNSUPPORTED;
+  if (!swap) { p.n1 = (int)(bi / 128); p.n3 = (int)(bo / n); }
+  else { p.n1 = (int)(bi / n); p.n3 = (int)(bo / 128); }
+  p.n2 = q;
+  return launch<true, true, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+}
+
+aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const aal_mat& Z,
+                     cudaStream_t s) {
+  if (!is_sm100()) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(X) || !tc_aligned(W) || !tc_aligned(Z)) return AAL_ERR_UNSUPPORTED;
+  const long long n = X.rows, b = n / q;
+  if (b % 128 || b > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.op = OP_SQUARE;
+  p.law = law;
+  p.q = q;
+  p.qv = 1;
+  p.bi = (int)b;
+  p.bo = (int)b;
+  p.out = (__nv_bfloat16*)Z.ptr;
+  p.ldo = Z.ld;
+  const int nn = pick_n(b, 256);
+  p.xr = 128;
+  p.wn = nn;
+  p.n_mma = nn;
+  p.a_rows = 128;
+  p.b_rows = nn;
+  p.b_aw = nn % 64 == 0 ? 64 : 16;
+  p.idesc = make_idesc(128, nn, false, true);
+  if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapA[0], X, 1, 128)) return AAL_ERR_UNSUPPORTED;
+  if (!map_mn(&p.mapB[0], W, 1, p.b_aw, nn, &p.b_merged)) return AAL_ERR_UNSUPPORTED;
+  if (!out_map(p, Z, 1)) return AAL_ERR_UNSUPPORTED;
+  p.n1 = (int)(b / 128);
+  p.n2 = q;
+  p.n3 = (int)(b / nn);
+  return launch<false, true, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
 }
 
 }  // namespace aal

@@ -214,6 +214,8 @@ AAL_API int32_t aal_last_path(void);
  * on this host thread only: the library records the CUDA event ``before``
  * (a cudaEvent_t) on the call's stream just before that launch and ``after``
  * just after it, then forgets both.  Passing NULL events clears the hook.
+ * During CUDA-graph capture the records become event-record nodes of the
+ * graph, so the events time the launch on every replay.
  * Kinds: AAL_KERNEL_PROJECT (1, also the down projection inside
  * aal_swiglu_fwd), AAL_KERNEL_GATE_UP (2, the fused gate/up/SiLU kernel of
  * aal_swiglu_fwd), AAL_KERNEL_BWD_DX (3), AAL_KERNEL_BWD_DW (4),

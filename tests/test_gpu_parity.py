@@ -65,9 +65,14 @@ def test_c1_all_calls_small(dtype):
 
 
 # ------------------------------------------------- Q2 x Q2 SwiGLU (110M FFN)
+TENSOR = aal.AAL_PATH_TENSOR
+
+
 def test_c2_swiglu_full_size():
+    # the launch configuration bench.py times (tensor-core path)
     eh, ey, path = run_swiglu("Q2xQ2", 4, 12288, 768, 1536, "bf16", seq_len=1536)
     assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+    assert path == TENSOR
 
 
 @pytest.mark.parametrize("B", [1, 8, 64])
@@ -89,15 +94,22 @@ def test_c2_decode_single_type(t):
 def test_c3_swiglu_full_size():
     eh, ey, path = run_swiglu("Q", 32, 2048, 4096, 12288, "bf16", seq_len=2048, w_sigma_rule="D")
     assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+    assert path == TENSOR
+
+
+def test_c3_projection_full_size():
+    err, path = run_project("Q", 32, 2048, 4096, 12288, "bf16", seq_len=2048)
+    assert err <= TOL["bf16"] and path == TENSOR, err
 
 
 # ------------------------------------------ Qwen3-30B-A3B-expert-shaped Q_16
 @pytest.mark.parametrize("din,dout", [(2048, 768), (768, 2048)])
 def test_c4_projection_fwd_bwd(din, dout):
-    err, _ = run_project("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
-    assert err <= TOL["bf16"], err
-    edx, edw, _ = run_bwd("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
+    err, path = run_project("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
+    assert err <= TOL["bf16"] and path == TENSOR, err
+    edx, edw, path = run_bwd("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
     assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
+    assert path == TENSOR
 
 
 def test_c4_swiglu():
@@ -114,6 +126,7 @@ def test_c5_square_full_size_sampled_tiles():
     Z = torch.empty_like(X)
     aal.aal_square_product("Q", q, X, W, Z)
     torch.cuda.synchronize()
+    assert aal.aal_last_path() == TENSOR
     Xh, Wh = ins["X"].t, ins["W"].t
     rng = np.random.default_rng(123)
     tiles = [(0, 0), (0, q - 1), (q - 1, 0), (q - 1, q - 1), (17, 17), (5, 200)]
@@ -132,8 +145,32 @@ def test_c5_square_full_size_sampled_tiles():
 
 @pytest.mark.parametrize("law,q,n", [("Q", 4, 512), ("Q", 16, 2048), ("Q2xQ2", 4, 256)])
 def test_square_medium(law, q, n):
-    err, _ = run_square(law, q, n, "bf16")
+    err, path = run_square(law, q, n, "bf16")
     assert err <= TOL["bf16"], err
+    assert path == (TENSOR if (n // q) % 128 == 0 else aal.AAL_PATH_GENERAL)
+
+
+@pytest.mark.parametrize("case", ["fwd_swap", "fwd_q2xq2", "swiglu_swap", "bwd_q4", "square_b256",
+                                  "fwd_offset", "fwd_ragged_tokens"])
+def test_tensor_path_small_cases(case):
+    T = TENSOR
+    if case == "fwd_swap":
+        r = run_project("Q", 8, 512, 1024, 1024, "bf16", seq_len=512, policy=T)
+    elif case == "fwd_q2xq2":
+        r = run_project("Q2xQ2", 4, 1024, 768, 1536, "bf16", seq_len=1024, policy=T)
+    elif case == "swiglu_swap":
+        eh, ey, p = run_swiglu("Q", 8, 512, 1024, 1024, "bf16", seq_len=512, policy=T)
+        r = (max(eh, ey), p)
+    elif case == "bwd_q4":
+        edx, edw, p = run_bwd("Q", 4, 512, 512, 512, "bf16", seq_len=512, policy=T)
+        r = (max(edx, edw), p)
+    elif case == "square_b256":
+        r = run_square("Q", 2, 512, "bf16", policy=T)
+    elif case == "fwd_offset":
+        r = run_project("Q", 8, 1024, 512, 1024, "bf16", seq_len=256, offset=5, policy=T)
+    else:  # tokens per class not a multiple of the 128-row tile
+        r = run_project("Q", 4, 4 * 200, 256, 512, "bf16", seq_len=800, policy=T)
+    assert r[0] <= TOL["bf16"] and r[1] == T, r
 
 
 # ---------------------------------------------------------------- edge cases
