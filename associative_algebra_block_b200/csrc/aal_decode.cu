@@ -13,6 +13,7 @@
 // scalar fallback.
 #include <cooperative_groups.h>
 #include <limits.h>
+#include <stdlib.h>
 
 #include "aal_internal.h"
 
@@ -463,6 +464,191 @@ static cudaError_t launch_split(const cudaLaunchConfig_t& cfg0, int cl, int law,
                             (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)x.cols, rows);
 }
 
+// Type-major variant (the default for aligned bf16 weights).  CTA (slab, t)
+// owns a 32-column slab inside output group k and the batch entries of row
+// type t: it gathers their indices, streams only the weight rows of the
+// groups in S(t, k) (agihunt.info digest, multiplication-table paragraph) and
+// computes the type's entries CH at a time from them, so no weight row is
+// read for an entry that does not use it.  The chunk's activations on those
+// rows are staged in shared memory as [row][entry] so that one weight row
+// feeds CH entries x 8 columns of FMAs from CH/8 128-bit shared loads.
+// Thread (cv, rl): cv = lane & 3 picks 8 of the 32 columns, rl =
+// (warp, lane >> 2) one of 64 row lanes; partial sums over the row lanes meet
+// through warp shuffles and shared memory.
+constexpr int kTmMaxB = 1024;    // batch entries scanned per CTA
+constexpr int kTmRound = 4;      // weight rows in flight per thread
+
+template <int CH>
+__global__ void __launch_bounds__(256)
+k_decode_typed(int law, int q, const int64_t* __restrict__ pos, int B,
+               const __nv_bfloat16* __restrict__ x, long long ldx,
+               const __nv_bfloat16* __restrict__ W, long long ldw, __nv_bfloat16* __restrict__ y,
+               long long ldy, int bi, int bo) {
+  constexpr int XS = CH < 8 ? 8 : CH;  // entries per staged row (padded to 16 bytes)
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(dsm);  // [needed row][XS]
+  __shared__ float red[8][CH][32];
+  __shared__ int s_idx[kTmMaxB];
+  __shared__ int s_wbase[8];
+  __shared__ int s_cnt;
+  __shared__ int s_grp[4];
+  __shared__ int s_ngrp;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cv = lane & 3, rl = warp * 8 + (lane >> 2);
+  const int col0 = blockIdx.x * 32, col = col0 + cv * 8;
+  const int k = col0 / bo;
+  const int t = blockIdx.y;
+
+  // 1. entries of type t (ballot compaction, order preserved)
+  if (tid == 0) s_cnt = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+    const int b = b0 + tid;
+    bool mine = false;
+    if (b < B) {
+      const long long p = pos[b];
+      if (p < 0) {
+        if (t == 0 && blockIdx.x == 0) flag_device_error(kDevBounds);
+      } else {
+        mine = (int)(p % q) == t;
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, mine);
+    if (lane == 0) s_wbase[warp] = __popc(m);
+    __syncthreads();
+    if (tid == 0) {
+      int acc = s_cnt;
+      for (int w = 0; w < 8; ++w) { const int c = s_wbase[w]; s_wbase[w] = acc; acc += c; }
+      s_cnt = acc;
+    }
+    __syncthreads();
+    if (mine) s_idx[s_wbase[warp] + __popc(m & ((1u << lane) - 1u))] = b;
+    __syncthreads();
+  }
+  const int cnt = s_cnt;
+  if (cnt == 0) return;
+  // 2. the groups this type needs for output group k
+  if (tid == 0) {
+    int mem[4];
+    s_ngrp = table_members(law, q, t, k, mem);
+    for (int i = 0; i < s_ngrp; ++i) s_grp[i] = mem[i];
+  }
+  __syncthreads();
+  const int ngrp = s_ngrp;
+  const int nvec = bi >> 3;  // 8-row pieces per group
+
+  for (int e0 = 0; e0 < cnt; e0 += CH) {
+    const int ne = min(CH, cnt - e0);
+    // 3. stage: item = (needed 8-row piece, entry); entries vary fastest
+    for (int i = tid; i < XS * ngrp * nvec; i += blockDim.x) {
+      const int e = i % XS, pv = i / XS, g = pv / nvec, r8 = (pv - g * nvec) * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (e < ne)
+        v = __ldg(reinterpret_cast<const uint4*>(x + (long long)s_idx[e0 + e] * ldx + s_grp[g] * bi + r8));
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&v);
+      __nv_bfloat16* d = xs + (size_t)(g * bi + r8) * XS + e;
+#pragma unroll
+      for (int m = 0; m < 8; ++m) d[m * XS] = h[m];
+    }
+    __syncthreads();
+    float acc[CH][8];
+#pragma unroll
+    for (int e = 0; e < CH; ++e)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[e][c] = 0.f;
+    for (int g = 0; g < ngrp; ++g) {
+      const __nv_bfloat16* wg = W + (long long)s_grp[g] * bi * ldw + col;
+      const __nv_bfloat16* xg = xs + (size_t)g * bi * XS;
+      for (int r0 = rl; r0 < bi; r0 += 64 * kTmRound) {
+        uint4 wv[kTmRound];
+#pragma unroll
+        for (int u = 0; u < kTmRound; ++u) {
+          const int r = r0 + 64 * u;
+          if (r < bi) wv[u] = __ldg(reinterpret_cast<const uint4*>(wg + (long long)r * ldw));
+        }
+#pragma unroll
+        for (int u = 0; u < kTmRound; ++u) {
+          const int r = r0 + 64 * u;
+          if (r >= bi) continue;
+          float w[8];
+          unpack16<__nv_bfloat16>(wv[u], w);
+          const uint4* xr = reinterpret_cast<const uint4*>(xg + (size_t)r * XS);
+#pragma unroll
+          for (int e8 = 0; e8 < (CH + 7) / 8; ++e8) {
+            float xf[8];
+            unpack16<__nv_bfloat16>(xr[e8], xf);
+#pragma unroll
+            for (int m = 0; m < 8 && e8 * 8 + m < CH; ++m)
+#pragma unroll
+              for (int c = 0; c < 8; ++c) acc[e8 * 8 + m][c] = fmaf(xf[m], w[c], acc[e8 * 8 + m][c]);
+          }
+        }
+      }
+    }
+    // 4. reduce over the 64 row lanes: shuffles over lane bits 2..4, then warps
+#pragma unroll
+    for (int e = 0; e < CH; ++e)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float v = acc[e][c];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        acc[e][c] = v;
+      }
+    if ((lane >> 2) == 0) {
+#pragma unroll
+      for (int e = 0; e < CH; ++e)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) red[warp][e][cv * 8 + c] = acc[e][c];
+    }
+    __syncthreads();
+    for (int i = tid; i < ne * 32; i += blockDim.x) {
+      const int e = i >> 5, cc = i & 31;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) sum += red[w][e][cc];
+      y[(long long)s_idx[e0 + e] * ldy + col0 + cc] = __float2bfloat16_rn(sum);
+    }
+    __syncthreads();  // xs and red are reused by the next chunk
+  }
+}
+
+template <int CH>
+static cudaError_t launch_typed(int law, int q, const int64_t* positions, int B, const aal_mat& x,
+                                const aal_mat& W, const aal_mat& y, int bi, int bo, long long dout,
+                                cudaStream_t s) {
+  constexpr int XS = CH < 8 ? 8 : CH;
+  const size_t xs_bytes = (size_t)4 * bi * XS * 2;  // at most 4 groups of bi rows
+  static unsigned long long attr_done = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_done & bit)) {
+    e = cudaFuncSetAttribute(k_decode_typed<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             160 * 1024);
+    if (e != cudaSuccess) return e;
+    attr_done |= bit;
+  }
+  dim3 grd((unsigned)(dout / 32), (unsigned)q);
+  k_decode_typed<CH><<<grd, 256, xs_bytes, s>>>(law, q, positions, B, (const __nv_bfloat16*)x.ptr,
+                                                x.ld, (const __nv_bfloat16*)W.ptr, W.ld,
+                                                (__nv_bfloat16*)y.ptr, y.ld, bi, bo);
+  return cudaGetLastError();
+}
+
+// AAL_DECODE_TYPED=0 in the environment selects the cluster kernel instead.
+static bool typed_disabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_DECODE_TYPED");
+    v = (e && e[0] == '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
                          const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled) {
   *handled = true;
@@ -472,11 +658,26 @@ aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat
   const int es = x.dtype == AAL_F32 ? 4 : 2, vec = 16 / es;
   const bool vec_ok = ((uintptr_t)W.ptr % 16) == 0 && W.ld % vec == 0 && bo % vec == 0 &&
                       x.cols <= INT_MAX && dout <= INT_MAX && B <= INT_MAX;
+  // type-major kernel: bf16, 32-column slabs inside one group, groups a
+  // multiple of 8 rows, at most 4 groups per table entry
+  if (vec_ok && x.dtype == AAL_BF16 && bo % 32 == 0 && bi % 8 == 0 && B <= kTmMaxB && q <= 65535 &&
+      x.ld % 8 == 0 && ((uintptr_t)x.ptr % 16) == 0 && (size_t)4 * bi * 16 * 2 <= 160 * 1024 &&
+      !typed_disabled() && (B <= 4 || B > 16 || bo % 64 != 0)) {
+    // measured on B200: the type-major kernel is fastest for small and large
+    // batches; between them the cluster kernel below is
+    cudaError_t e;
+    if (B <= 1) e = launch_typed<1>(law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else if (B <= 2) e = launch_typed<2>(law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else if (B <= 4) e = launch_typed<4>(law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else if (B <= 16) e = launch_typed<8>(law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else e = launch_typed<16>(law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    note_launch();
+    return cuda_status(e);
+  }
   // fp32 stays on the exact vector path below
   if (vec_ok && x.dtype == AAL_BF16 && bo % 64 == 0) {
     int cl = 1;
     while (cl < 8 && (x.cols + cl - 1) / cl > kMaxRowsCta) cl <<= 1;
-    while (cl < 8 && (x.cols + cl - 1) / cl > 96) cl <<= 1;  // shorter row ranges
     const int rows = (int)(((x.cols + cl - 1) / cl + 7) / 8 * 8);
     if (rows <= kMaxRowsCta && x.cols % 8 == 0 && x.ld % 8 == 0 && ((uintptr_t)x.ptr % 16) == 0 &&
         (B + 7) / 8 <= 65535) {
