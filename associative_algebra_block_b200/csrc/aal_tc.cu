@@ -18,10 +18,11 @@
 // [M/q][q][d]; a box with extent 1 in the middle dimension pulls the rows of
 // one type class straight out of HBM.  No index buffer, no copy.
 //
-// Roles (320 threads): warp 0 issues TMA loads, warp 1 owns TMEM and issues
-// the MMAs (one thread), warps 2..9 drain TMEM to registers and write bf16
-// results (optionally applying SiLU(g)*u or adding into the destination); two
-// epilogue warps share each 32-lane quarter of TMEM and split its columns.
+// Roles (416 threads): warps 0 and 10..12 issue TMA loads (chunk i goes to
+// producer warp i mod 4), warp 1 owns TMEM and issues the MMAs (one thread),
+// warps 2..9 drain TMEM to registers and write bf16 results (optionally
+// applying SiLU(g)*u or adding into the destination); two epilogue warps share
+// each 32-lane quarter of TMEM and split its columns.
 // Tiles are visited longest first: a tile's cost is the number of block
 // products in its table entry (1, 2 or 4 for the laws here, up to q for the
 // backward's diagonal blocks), and the persistent CTAs stride through the
@@ -40,7 +41,11 @@ namespace aal {
 namespace tc {
 
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+// TMA producer warps: warp 0 and the warps after the epilogue.  One warp's
+// bulk-tensor copies are issued one after another at several hundred cycles
+// each whatever the box size, so consecutive K chunks go to different warps.
+constexpr int kProdWarps = 4;
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * (kProdWarps - 1);
 constexpr int kMaxPairs = 256;
 constexpr int kMaxStages = 8;
 constexpr int kSmemBudget = 200 * 1024;
@@ -350,17 +355,54 @@ __device__ __forceinline__ uint64_t operand_kstep(int aw) {
 
 
 // ------------------------------------------------------------- tile layout
+// A tile description lives in registers: every access to its segment array
+// uses a constant index (a runtime index would put it in local memory, and
+// every role decodes every tile it visits).
 __device__ __forceinline__ void add_seg(TileDesc& d, int k0, int len, int cls, int map) {
   // merge with the previous segment when the K ranges touch (same class/map)
-  if (d.nseg > 0) {
-    Seg& s = d.seg[d.nseg - 1];
-    if (s.cls == cls && s.map == map && s.k0 + s.len == k0) { s.len += len; return; }
+  bool merged = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    Seg& s = d.seg[j];
+    if (j == d.nseg - 1 && s.cls == cls && s.map == map && s.k0 + s.len == k0) {
+      s.len += len;
+      merged = true;
+    }
   }
-  d.seg[d.nseg].k0 = k0;
-  d.seg[d.nseg].len = len;
-  d.seg[d.nseg].cls = cls;
-  d.seg[d.nseg].map = map;
+  if (merged) return;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (j == d.nseg) {
+      d.seg[j].k0 = k0;
+      d.seg[j].len = len;
+      d.seg[j].cls = cls;
+      d.seg[j].map = map;
+    }
+  }
   ++d.nseg;
+}
+__device__ __forceinline__ Seg seg_at(const TileDesc& d, int s) {
+  Seg r = d.seg[0];
+  if (s == 1) r = d.seg[1];
+  if (s == 2) r = d.seg[2];
+  if (s == 3) r = d.seg[3];
+  return r;
+}
+// The members a of S(t, k) in ascending order, each added as a K segment of
+// width ``w`` starting at a * w (class ``cls``).
+__device__ __forceinline__ void add_members(const Params& p, TileDesc& d, int t, int k, int w, int cls) {
+  if (p.law == AAL_LAW_Q) {
+    if (t == k) {
+      add_seg(d, t * w, w, cls, 0);
+    } else {
+      add_seg(d, min(t, k) * w, w, cls, 0);
+      add_seg(d, max(t, k) * w, w, cls, 0);
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      if (in_table(p.law, t, k, g)) add_seg(d, g * w, w, cls, 0);
+  }
 }
 
 // The p1 that makes pair (p0, p1) diagonal: the row type of class p0 for the
@@ -411,9 +453,7 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     case OP_FWD:
     case OP_SWIGLU: {  // i0 class, i1 token block, i2 output group k, i3 column block
       const int c = i0, k = i2, t = type_of_class(p, c);
-      int mem[4];
-      const int n = table_members(p.law, p.q, t, k, mem);
-      for (int s = 0; s < n; ++s) add_seg(d, mem[s] * p.bi, p.bi, c, 0);
+      add_members(p, d, t, k, p.bi, c);
       const int xrow0 = i1 * p.xr, wcol0 = k * p.bo + i3 * p.wn;
       if (!p.swap) { d.a_f = xrow0; d.a_c1 = 1; d.b_f = wcol0; d.b_c1 = 0; }
       else { d.a_f = wcol0; d.a_c1 = 0; d.b_f = xrow0; d.b_c1 = 1; }
@@ -422,9 +462,7 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     }
     case OP_SQUARE: {  // i0 row block i, i1 128-row slab, i2 column block k, i3 column slab
       const int i = i0, k = i2;
-      int mem[4];
-      const int n = table_members(p.law, p.q, i, k, mem);
-      for (int s = 0; s < n; ++s) add_seg(d, mem[s] * p.bi, p.bi, 0, 0);
+      add_members(p, d, i, k, p.bi, 0);
       d.a_f = i * p.bi + i1 * 128; d.a_c1 = 0;
       d.b_f = k * p.bo + i3 * p.wn; d.b_c1 = 0;
       d.rbase = d.a_f; d.cbase = d.b_f;
@@ -517,19 +555,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------ TMA producers
+    // Every producer warp walks the same chunk sequence and issues the chunks
+    // i with i mod nprod == its index.  With nprod <= S a warp waiting for
+    // stage i mod S to empty cannot mistake an older phase for the one it
+    // needs: its previous chunk i - nprod already saw chunk i - nprod - S
+    // released, and the MMAs release stages in order.
+    const int nprod = S < kProdWarps ? S : kProdWarps;
+    const int pw = warp == 0 ? 0 : warp - (1 + kEpiWarps);
     uint32_t it = 0, st = 0, ph = 0;
-    bool ok = true;
+    bool ok = pw < nprod;
     for (int tile = tile0; tile < p.ntiles && ok; tile += tstep) {
       TileDesc d;
       describe(p, tile, d);
       for (int s = 0; s < d.nseg && ok; ++s) {
-        const Seg sg = d.seg[s];
+        const Seg sg = seg_at(d, s);
         const int nch = seg_chunks(sg);
         for (int kc = 0; kc < nch; ++kc) {
-          if (!warp_wait(&empty_bar[st], ph ^ 1u, &s_abort)) { ok = false; break; }
-          {
+          const bool mine = (int)(it % (uint32_t)nprod) == pw;
+          if (mine && !warp_wait(&empty_bar[st], ph ^ 1u, &s_abort)) { ok = false; break; }
+          if (mine) {
             // The boxes of a stage are issued by separate lanes: one thread
             // issuing them back to back serialises the TMA requests.
             const uint32_t base = smem0 + st * p.stage_bytes;
@@ -588,8 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       }
     }
     // let every copy this CTA issued land before the CTA can exit (for a pair
-    // the pair's first CTA sees both halves on its own barriers)
-    if (lane == 0 && issuer) {
+    // the pair's first CTA sees both halves on its own barriers); warp 0 counts
+    // every chunk, so it waits for the last use of each stage
+    if (warp == 0 && lane == 0 && issuer) {
       for (int st = 0; st < S; ++st) {
         if ((uint32_t)st >= it) break;
         const uint32_t last = st + ((it - 1 - st) / S) * S;
@@ -628,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
         const uint32_t acc1 = acc0 + p.n_mma;
         uint32_t accumulate = 0;
         for (int s = 0; s < d.nseg && ok; ++s) {
-          const int len = d.seg[s].len;
+          const int len = seg_at(d, s).len;
           for (int rem = len; rem > 0; rem -= 64) {
             if (!(mbar_try_wait(&full_bar[st], ph) || mbar_wait(&full_bar[st], ph, &s_abort))) {
               ok = false;
@@ -684,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       else tc_commit(&done_bar);
       mbar_wait_teardown(&done_bar, 0);
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // ------------------------------------------------------ epilogue
     const int quarter = warp & 3;             // TMEM lanes this warp may read
     const int half = (warp - 2) / 4;          // which of the 16-column chunks it drains
