@@ -639,6 +639,280 @@ static cudaError_t launch_typed(int law, int q, const int64_t* positions, int B,
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------------------
+// Tensor-core decode.  A decode batch is a skinny product Y = X W in which
+// entry b may only use the weight blocks (a, k) with a in S(t_b, k)
+// (agihunt.info digest, multiplication-table paragraph and Transformer-mapping
+// paragraph).  Writing it as a dense product whose activations are zeroed
+// where the table says "not used" turns it into warp-level tensor-core MMAs
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate); the weight blocks that no
+// entry of the batch needs are neither loaded nor multiplied, so HBM traffic
+// stays the table's.  CTA (column tile, z) owns 64 output columns (inside one
+// output group k) and the K slice z of the weight rows; the slices of one
+// column tile form a thread-block cluster and their fp32 partial products
+// meet in distributed shared memory, each CTA summing and writing a share of
+// the batch rows.
+// Operand orientation: the MMA's M is the 64 output columns (A = W^T, read
+// from the row-major weight tile with ldmatrix .trans), N the batch entries
+// (B = X^T, rows of X), K the weight rows.
+constexpr int kMmaCols = 64;      // output columns per CTA
+constexpr int kMmaMaxB = 256;     // batch entries per launch
+constexpr int kMmaKc = 192;       // weight rows staged per round
+constexpr int kMmaWStride = 72;   // staged weight row: 64 columns + 8 pad (144 bytes)
+constexpr int kMmaPStride = 68;   // fp32 partial row: 64 columns + 4 pad
+
+__device__ __forceinline__ uint32_t dec_smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  // src_bytes 0 fills the 16 bytes with zeros
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// NT: n-tiles (8 entries) per warp; warps 0..3 take the four 16-column
+// m-tiles, warps 4..7 the same m-tiles for the odd n-tiles.
+// Latency is the cost at these sizes, so the first round's copies start
+// before the row types are known: the weight rows of the whole round are
+// fetched (later rounds fetch only the groups some entry uses), the
+// activations unmasked, and an entry's table row is applied to its operand
+// fragment in registers.
+template <int NT>
+__global__ void __launch_bounds__(256)
+k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
+             const __nv_bfloat16* __restrict__ x, long long ldx,
+             const __nv_bfloat16* __restrict__ W, long long ldw, __nv_bfloat16* __restrict__ y,
+             long long ldy, int bi, int bo, int slice) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __shared__ int s_type[kMmaMaxB];
+  __shared__ unsigned long long s_present;
+  __shared__ unsigned char s_used[64];  // groups of the CTA's K slice that some entry uses
+  cg::cluster_group cluster = cg::this_cluster();
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = blockIdx.x * kMmaCols;
+  const int k = c0 / bo;
+  const int ks0 = blockIdx.z * slice;  // first weight row of this CTA
+  const int Bp = (B + 7) & ~7;
+  const int ntiles = Bp >> 3;
+  const int xs_stride = kMmaKc + 8;  // staged activation row, bf16
+  __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(dsm);
+  __nv_bfloat16* Xs = Ws + kMmaKc * kMmaWStride;
+  float* P = reinterpret_cast<float*>(dsm);  // reused after the MMAs
+  const int g0 = ks0 / bi, ng = (ks0 + slice - 1) / bi - g0 + 1;
+
+  auto stage = [&](int r0, int rows, bool all_rows) {
+    for (int i = tid; i < rows * 8; i += blockDim.x) {
+      const int r = i >> 3, ch = i & 7;
+      if (all_rows || s_used[(r0 + r) / bi - g0])
+        cp_async16(dec_smem_u32(Ws + r * kMmaWStride + ch * 8),
+                   W + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
+    }
+    const int xch = rows >> 3;
+    for (int i = tid; i < Bp * xch; i += blockDim.x) {
+      const int n = i / xch, ch = i - n * xch;
+      const bool in = n < B;
+      cp_async16(dec_smem_u32(Xs + n * xs_stride + ch * 8),
+                 in ? x + (long long)n * ldx + r0 + ch * 8 : x, in ? 16u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  // round 0's copies go out first
+  stage(ks0, min(kMmaKc, slice), true);
+
+  // 1. row type of every entry; -1 for padding and invalid positions
+  if (tid == 0) s_present = 0ull;
+  __syncthreads();
+  for (int b = tid; b < Bp; b += blockDim.x) {
+    int t = -1;
+    if (b < B) {
+      const long long p = pos[b];
+      if (p < 0) {
+        if (blockIdx.x == 0 && blockIdx.z == 0) flag_device_error(kDevBounds);
+      } else {
+        t = (int)(p % q);
+        atomicOr(&s_present, 1ull << t);
+      }
+    }
+    s_type[b] = t;
+  }
+  __syncthreads();
+  // 2. which groups a of the slice some present type uses with output group k
+  if (tid < ng) {
+    const int a = g0 + tid;
+    const unsigned long long pres = s_present;
+    bool u = false;
+    for (int t = 0; t < q && !u; ++t)
+      if ((pres >> t) & 1ull) u = in_table(law, t, k, a);
+    s_used[tid] = u ? 1 : 0;
+  }
+
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+  const int mt = warp & 3, nt0 = warp >> 2;
+  const int g = lane >> 2;
+  // row types of the entries whose B fragments this thread holds
+  int my_t[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int n = (nt0 + 2 * j) * 8 + g;
+    my_t[j] = n < Bp ? s_type[n] : -1;
+  }
+
+  for (int kc = 0; kc < slice; kc += kMmaKc) {
+    const int rows = min(kMmaKc, slice - kc);
+    const int r0 = ks0 + kc;  // first weight row of this round
+    if (kc > 0) stage(r0, rows, false);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    // 3. MMAs over the used 16-row steps; an entry whose table row does not
+    //    use the step's group contributes zeros
+    int a_prev = -1;
+    unsigned keep = 0;  // bit j: entry of n-tile j uses group a
+    for (int kk = 0; kk < rows; kk += 16) {
+      const int a = (r0 + kk) / bi;
+      if (!s_used[a - g0]) continue;
+      if (a != a_prev) {
+        keep = 0;
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          if (my_t[j] >= 0 && in_table(law, my_t[j], k, a)) keep |= 1u << j;
+        a_prev = a;
+      }
+      uint32_t af[4];
+      const int arow = kk + (lane & 7) + ((lane >> 4) << 3);
+      const int acol = mt * 16 + (((lane >> 3) & 1) << 3);
+      ldsm_x4_trans(dec_smem_u32(Ws + arow * kMmaWStride + acol), af);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const int nt = nt0 + 2 * j;
+        if (nt < ntiles) {
+          uint32_t bf[2];
+          const int brow = nt * 8 + (lane & 7);
+          const int bcol = kk + (((lane >> 3) & 1) << 3);
+          ldsm_x2(dec_smem_u32(Xs + brow * xs_stride + bcol), bf);
+          if (!((keep >> j) & 1u)) { bf[0] = 0u; bf[1] = 0u; }
+          mma_bf16_16816(acc[j], af, bf);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // 4. fp32 partials [entry][column] in shared memory
+  const int c = lane & 3;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int nt = nt0 + 2 * j;
+    if (nt < ntiles) {
+      const int n = nt * 8 + 2 * c, m = mt * 16 + g;
+      P[n * kMmaPStride + m] = acc[j][0];
+      P[(n + 1) * kMmaPStride + m] = acc[j][1];
+      P[n * kMmaPStride + m + 8] = acc[j][2];
+      P[(n + 1) * kMmaPStride + m + 8] = acc[j][3];
+    }
+  }
+  cluster.sync();
+  // 5. CTA z sums rows z, z + cl, ... over the cluster (4 columns per thread,
+  //    every peer's load in flight at once) and writes them
+  const int cl = (int)gridDim.z, z = (int)blockIdx.z;
+  const int my_rows = (Bp - z + cl - 1) / cl;
+  for (int i = tid; i < my_rows * 16; i += blockDim.x) {
+    const int n = z + cl * (i >> 4), ch = i & 15;
+    if (n >= B || s_type[n] < 0) continue;
+    float4 u[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < cl)
+        u[r] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(P, r) + n * kMmaPStride + ch * 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < cl) { v.x += u[r].x; v.y += u[r].y; v.z += u[r].z; v.w += u[r].w; }
+    uint2 o;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+    h[0] = __floats2bfloat162_rn(v.x, v.y);
+    h[1] = __floats2bfloat162_rn(v.z, v.w);
+    *reinterpret_cast<uint2*>(y + (long long)n * ldy + c0 + ch * 4) = o;
+  }
+  cluster.sync();  // no CTA leaves while a peer still reads its partials
+}
+
+static size_t mma_smem_bytes(int Bp) {
+  const size_t stage = (size_t)kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
+  const size_t part = (size_t)Bp * kMmaPStride * 4;
+  return stage > part ? stage : part;
+}
+
+template <int NT>
+static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, int B,
+                              const aal_mat& x, const aal_mat& W, const aal_mat& y, int bi, int bo,
+                              long long dout, cudaStream_t s) {
+  const int Bp = (B + 7) & ~7;
+  const size_t smem = mma_smem_bytes(Bp);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static unsigned long long attr_done = 0;  // per device (bit dev % 64)
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_done & bit)) {
+    e = cudaFuncSetAttribute(k_decode_mma<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)mma_smem_bytes(kMmaMaxB));
+    if (e != cudaSuccess) return e;
+    attr_done |= bit;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(dout / kMmaCols), 1, (unsigned)cl);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = cl;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_decode_mma<NT>, law, q, positions, B,
+                            (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr, W.ld,
+                            (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)(x.cols / cl));
+}
+
+static bool aligned16(const aal_mat& m) {
+  return ((uintptr_t)m.ptr % 16) == 0 && m.ld % 8 == 0;
+}
+
+// AAL_DECODE_MMA=0 in the environment turns the tensor-core decode off.
+static bool mma_disabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_DECODE_MMA");
+    v = (e && e[0] == '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
 // AAL_DECODE_TYPED=0 in the environment selects the cluster kernel instead.
 static bool typed_disabled() {
   static int v = -1;
@@ -658,6 +932,20 @@ aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat
   const int es = x.dtype == AAL_F32 ? 4 : 2, vec = 16 / es;
   const bool vec_ok = ((uintptr_t)W.ptr % 16) == 0 && W.ld % vec == 0 && bo % vec == 0 &&
                       x.cols <= INT_MAX && dout <= INT_MAX && B <= INT_MAX;
+  // tensor-core kernel: bf16, 64-column tiles inside one output group,
+  // 16-row steps inside one input group, at most 256 entries
+  if (x.dtype == AAL_BF16 && W.dtype == AAL_BF16 && y.dtype == AAL_BF16 && B <= kMmaMaxB &&
+      q <= 64 && bo % kMmaCols == 0 && bi % 16 == 0 && aligned16(x) && aligned16(W) &&
+      aligned16(y) && x.cols <= INT_MAX && dout <= INT_MAX && !mma_disabled()) {
+    int cl = 8;
+    while (cl > 1 && (x.cols % (16 * cl)) != 0) cl >>= 1;
+    cudaError_t e;
+    if (B <= 16) e = launch_mma<1>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else if (B <= 64) e = launch_mma<4>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    else e = launch_mma<16>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    note_launch();
+    return cuda_status(e);
+  }
   // type-major kernel: bf16, 32-column slabs inside one group, groups a
   // multiple of 8 rows, at most 4 groups per table entry
   if (vec_ok && x.dtype == AAL_BF16 && bo % 32 == 0 && bi % 8 == 0 && B <= kTmMaxB && q <= 65535 &&

@@ -36,6 +36,27 @@ from associative_algebra_block_b200 import inputs  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
+# capture of this command on a B200 (summaries under profiles/).  A figure is
+# used only while the tensor-core source still hashes to the value it was
+# taken with; after any change to the kernel the bench reports null.
+NCU_TRAFFIC = {
+    # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
+}
+
+
+def _kernel_sha(source):
+    import hashlib
+    with open(os.path.join(ROOT, "associative_algebra_block_b200", "csrc", source), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def _traffic(config, kernel):
+    rec = NCU_TRAFFIC.get((config, kernel))
+    if rec is None or rec[0] != _kernel_sha(rec[2]):
+        return None
+    return rec[1]
+
 
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -50,6 +71,14 @@ def _peaks():
 # ---------------------------------------------------------------------------
 # Workloads
 # ---------------------------------------------------------------------------
+
+def _marker(ev):
+    """mark(j) arms timing slot j's event pair (if it has one) for the next
+    launch of its kind."""
+    if ev is None:
+        return lambda j: None
+    return lambda j: ev[j] is not None and aal.aal_set_timing_events(ev[j][0], ev[j][1], ev[j][2])
+
 
 def _exec_flops_proj(law, q, M, din, dout):
     per_row = aal.aal_block_product_count(law, q, True)
@@ -70,9 +99,6 @@ class SwigluDecode:
                              for B in decode_batches)
         self.exec_flops = self.fwd_flops + self.dec_flops
         self.dense_flops = 2 * M * D * F * 3 + sum(2 * B * D * F * 3 for B in decode_batches)
-        self.dominant = aal.AAL_KERNEL_GATE_UP
-        self.dominant_flops = self.gate_up_flops
-        self.dominant_name = "gate_up (fused gate/up projections + SiLU*mul)"
 
     def config(self):
         return {"workload": f"{self.name}: {self.law} q={self.q} SwiGLU FFN fwd d={self.D} "
@@ -118,15 +144,48 @@ class SwigluDecode:
                                   y=torch.empty_like(d["y"], device="cpu").pin_memory())
                              for d in self.sets[0]["dec"]])
 
+    def kernel_model(self, name, sets):
+        """(FLOPs, algorithmic bytes) of one launch of kernel ``name``."""
+        M, D, F, e = self.M, self.D, self.F, 2
+        if name == "gate_up":
+            return self.gate_up_flops, e * (M * D + 2 * D * F + M * F)
+        if name == "down":
+            return _exec_flops_proj(self.law, self.q, M, F, D), e * (M * F + D * F + M * D)
+        B = int(name.split("=")[1])
+        k = self.decode_batches.index(B)
+        pos = sets[0]["dec"][k]["pos"].cpu().numpy()
+        types = sorted(set(int(t) for t in pos % self.q))
+        S = aal.aal_block_table(self.law, self.q)
+        used = sum(1 for kk in range(self.q) for a in range(self.q) if any(S[t, kk, a] for t in types))
+        flops, byts = 0, 0
+        for din, dout in ((D, F), (D, F), (F, D)):
+            bi, bo = din // self.q, dout // self.q
+            n_blocks = sum(int(S[int(t) % self.q, kk, a]) for t in pos for kk in range(self.q) for a in range(self.q))
+            flops += 2 * bi * bo * n_blocks
+            byts += e * (used * bi * bo + B * (din + dout)) + 8 * B
+        return flops / 3, byts / 3  # mean over the three projections of a decode step
+
+    def timing_slots(self):
+        """(name, kernel kind) of every launch of a step, in launch order;
+        launches that share a name are one kernel of the breakdown."""
+        slots = [("gate_up", aal.AAL_KERNEL_GATE_UP), ("down", aal.AAL_KERNEL_PROJECT)]
+        for B in self.decode_batches:
+            slots += [(f"decode B={B}", aal.AAL_KERNEL_DECODE)] * 3
+        return slots
+
     def step(self, i, ev=None):
+        """``ev``: None, or one (before, after) event pair per timing slot."""
         s = self.sets[i % len(self.sets)]
-        if ev is not None:
-            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
+        mark = _marker(ev)
+        mark(0)
+        mark(1)
         aal.aal_swiglu_fwd(self.law, self.q, self.rule, s["X"], s["Wg"], s["Wu"], s["Wd"], s["H"], s["Y"])
+        j = 2
         for d in s["dec"]:
-            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["x"], s["Wg"], d["g"])
-            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["x"], s["Wu"], d["u"])
-            aal.aal_decode_matvec(self.law, self.q, d["pos"], d["h"], s["Wd"], d["y"])
+            for x, w, y in ((d["x"], s["Wg"], d["g"]), (d["x"], s["Wu"], d["u"]), (d["h"], s["Wd"], d["y"])):
+                mark(j)
+                aal.aal_decode_matvec(self.law, self.q, d["pos"], x, w, y)
+                j += 1
 
     def dense_step(self, i):
         s = self.sets[i % len(self.sets)]
@@ -197,9 +256,6 @@ class ProjFwdBwd:
         f2 = _exec_flops_proj(law, q, M, F, D)
         self.exec_flops = 3 * (f1 + f2)
         self.dense_flops = 3 * 2 * (2 * M * D * F)
-        self.dominant = aal.AAL_KERNEL_PROJECT
-        self.dominant_flops = f1
-        self.dominant_name = "project (D->F)"
 
     def config(self):
         return {"workload": f"{self.name}: {self.law} q={self.q} projections {self.D}->{self.F} and "
@@ -224,12 +280,27 @@ class ProjFwdBwd:
             self.sets.append(s)
         self.rule = aal.row_rule(seq_len=self.seq_len)
 
+    def kernel_model(self, name, sets):
+        kind, shape = name.rsplit(" ", 1)
+        din, dout = (int(v) for v in shape.split("->"))
+        f = _exec_flops_proj(self.law, self.q, self.M, din, dout)
+        return f, 2 * (self.M * din + din * dout + self.M * dout)
+
+    def timing_slots(self):
+        out = []
+        for t in (f"{self.D}->{self.F}", f"{self.F}->{self.D}"):
+            out += [(f"project {t}", aal.AAL_KERNEL_PROJECT), (f"bwd dX {t}", aal.AAL_KERNEL_BWD_DX),
+                    (f"bwd dW {t}", aal.AAL_KERNEL_BWD_DW)]
+        return out
+
     def step(self, i, ev=None):
         s = self.sets[i % len(self.sets)]
-        if ev is not None:
-            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
-        for t in ("a", "b"):
+        mark = _marker(ev)
+        for n, t in enumerate(("a", "b")):
+            mark(3 * n)
             aal.aal_project_fwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "Y"])
+            mark(3 * n + 1)
+            mark(3 * n + 2)
             aal.aal_project_bwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "dY"],
                                 s[t + "dX"], s[t + "dW"])
 
@@ -249,9 +320,6 @@ class Square:
         b = n // q
         self.exec_flops = 2 * aal.aal_block_product_count(law, q, False) * b ** 3
         self.dense_flops = 2 * n ** 3
-        self.dominant = aal.AAL_KERNEL_SQUARE
-        self.dominant_flops = self.exec_flops
-        self.dominant_name = "square product"
 
     def config(self):
         return {"workload": f"{self.name}: square product {self.law} q={self.q} n={self.n} b={self.n // self.q}",
@@ -267,10 +335,15 @@ class Square:
             self.n ** -0.5).to(torch.bfloat16)
         self.sets = [dict(X=X, W=W, Z=torch.empty_like(X))]
 
+    def kernel_model(self, name, sets):
+        return self.exec_flops, 3 * self.n * self.n * 2
+
+    def timing_slots(self):
+        return [("square product", aal.AAL_KERNEL_SQUARE)]
+
     def step(self, i, ev=None):
         s = self.sets[0]
-        if ev is not None:
-            aal.aal_set_timing_events(self.dominant, ev[0], ev[1])
+        _marker(ev)(0)
         aal.aal_square_product(self.law, self.q, s["X"], s["W"], s["Z"])
 
     def dense_step(self, i):
@@ -355,12 +428,21 @@ def _barrier(dist_on):
     torch.cuda.synchronize()
 
 
-def _max_over_ranks(v, dist_on):
+def _max_over_ranks(v, dist_on, device="cuda"):
+    """The slowest rank's value (the job ends when its last rank does)."""
     if not dist_on:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(total_ms_max, steps, world, flops_per_rank_step):
+    """Whole-job TFLOP/s: every rank runs the same per-GPU step on its own
+    tokens, so the job does ``world`` times the per-rank work in the slowest
+    rank's time."""
+    ms = total_ms_max / steps
+    return world * flops_per_rank_step / (ms * 1e-3) / 1e12, ms
 
 
 def time_steps(fn, steps, warmup, dist_on):
@@ -378,24 +460,35 @@ def time_steps(fn, steps, warmup, dist_on):
     return start.elapsed_time(stop)
 
 
-def capture_steps(step, nsets, with_events):
-    """One CUDA graph per rotating input set, each holding one whole step.
-    With ``with_events`` the dominant kernel's launch is bracketed by a pair of
-    events captured into the graph (record nodes), one pair per set."""
-    evs = []
-    for _ in range(nsets):
+def make_events(slots, only=None):
+    """One (kind, before, after) triple per timing slot (None for the slots
+    not named ``only`` when it is given)."""
+    out = []
+    for name, kind in slots:
+        if only is not None and name != only:
+            out.append(None)
+            continue
         a = torch.cuda.Event(enable_timing=True, external=True)
         b = torch.cuda.Event(enable_timing=True, external=True)
         a.record()  # torch creates the CUDA event on first record
         b.record()
-        evs.append((a, b))
+        out.append((kind, a, b))
+    return out
+
+
+def capture_steps(step, nsets, slots, only=None):
+    """One CUDA graph per rotating input set, each holding one whole step.
+    With ``slots`` the launches of the step (those named ``only``, if given)
+    are bracketed by pairs of events captured into the graph (record nodes),
+    one set of pairs per graph."""
+    evs = [make_events(slots, only) for _ in range(nsets)] if slots else [None] * nsets
     torch.cuda.synchronize()
     graphs = []
     side = torch.cuda.Stream()
     for i in range(nsets):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
-            step(i, evs[i] if with_events else None)
+            step(i, evs[i])
         graphs.append(g)
     torch.cuda.synchronize()
     return graphs, evs
@@ -458,7 +551,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-rows", type=int, default=768)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--launch", default="eager", choices=["eager", "graph"],
+    ap.add_argument("--launch", default="graph", choices=["eager", "graph"],
                     help="timed region: eager calls through the binding, or CUDA-graph replay")
     args = ap.parse_args()
 
@@ -493,27 +586,48 @@ def main():
         raise SystemExit("device status not ok after the eager pass")
 
     # ---- timed region: K steps of the whole path
+    # ---- per-kernel breakdown (before the timed region): every launch of a
+    # step bracketed by CUDA events on its stream.  An event pair adds a few
+    # microseconds to what it brackets, so the timed region below brackets
+    # only the launches of the kernel with the largest share.
+    slots = wl.timing_slots()
+    if args.launch == "graph":
+        bgraphs, bevs = capture_steps(wl.step, nsets, slots)
+        for _ in range(max(3, args.warmup)):
+            for g in bgraphs:
+                g.replay()
+        torch.cuda.synchronize()
+        del bgraphs
+    else:
+        bevs = []
+        for i in range(max(3, args.warmup) * nsets):
+            ev = make_events(slots)
+            wl.step(i, ev)
+            bevs.append(ev)
+        torch.cuda.synchronize()
+    per = {}
+    for ev in bevs:
+        for (name, _), (_, a, b) in zip(slots, ev):
+            per.setdefault(name, []).append(a.elapsed_time(b))
+    nper = {name: sum(1 for n, _ in slots if n == name) for name in per}
+    dom = max(per, key=lambda n: statistics.mean(per[n]) * nper[n])
+
     aal.aal_launch_count(reset=True)
     if args.launch == "graph":
-        graphs, evs = capture_steps(wl.step, nsets, with_events=True)
+        # the events of graph g time the dominant kernel in g's last replay
+        graphs, evs = capture_steps(wl.step, nsets, slots, only=dom)
         launches_per_step = aal.aal_launch_count(reset=True) / nsets
         run_step = lambda i: graphs[i % nsets].replay()
     else:
         graphs = None
-        evs = []
-        for _ in range(args.steps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()  # torch creates the CUDA event on first record
-            b.record()
-            evs.append((a, b))
+        evs = [make_events(slots, only=dom) for _ in range(args.steps)]
         torch.cuda.synchronize()
         wl.step(0)  # one step to count launches
         torch.cuda.synchronize()
         launches_per_step = aal.aal_launch_count(reset=True)
-        step_no = [0]
 
         def run_step(i):
-            # the events of timed step t bracket the dominant kernel's launch
+            # timed step t records its own events around the dominant kernel
             t = i - args.warmup
             wl.step(i, evs[t] if 0 <= t < len(evs) else None)
     with ClockSampler(torch.cuda.current_device()) as clk:
@@ -522,24 +636,42 @@ def main():
     if status != aal.AAL_OK:
         raise SystemExit(f"device status after the timed region: {aal.status_string(status)}")
     total_ms = _max_over_ranks(total_ms, dist_on)
-    ms = total_ms / args.steps
-    value = world * wl.exec_flops / (ms * 1e-3) / 1e12
+    value, ms = job_throughput(total_ms, args.steps, world, wl.exec_flops)
 
-    # ---- dominant kernel: CUDA events recorded on the launching stream right
-    # before and after its launch, inside the timed region
-    kern = [a.elapsed_time(b) for a, b in evs]
-    kms = statistics.mean(kern)
-    achieved = wl.dominant_flops / (kms * 1e-3) / 1e12
+    # the dominant kernel inside the timed region
+    live = [e[1].elapsed_time(e[2]) for ev in evs for e in ev if e is not None]
+    breakdown = {}
+    for name, v in per.items():
+        launch_ms = statistics.mean(live) if name == dom else statistics.mean(v)
+        flops, byts = wl.kernel_model(name, wl.sets)
+        breakdown[name] = {"launches_per_step": nper[name], "ms_per_launch": launch_ms,
+                           "share_of_step": launch_ms * nper[name] / ms,
+                           "tflops": flops / (launch_ms * 1e-3) / 1e12,
+                           "gbs": byts / (launch_ms * 1e-3) / 1e9,
+                           "flops_per_launch": flops, "bytes_per_launch": byts,
+                           "timed": "live, inside the timed region" if name == dom
+                                    else "breakdown pass before the timed region"}
+    dk = breakdown[dom]
     long_region = total_ms > 2000.0
-    peak = peaks["bf16_sust"] if long_region else peaks["bf16"]
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
-                "kernel": wl.dominant_name, "kernel_ms": kms,
-                "kernel_share_of_step": kms / ms,
-                "peak_kind": ("sustained" if long_region else "burst") + f" bf16, {peaks['source']}"}
+    peak_t = peaks["bf16_sust"] if long_region else peaks["bf16"]
+    ridge = peak_t * 1e12 / (peaks["hbm"] * 1e9)
+    bound = "tensor" if dk["flops_per_launch"] / dk["bytes_per_launch"] > ridge else "hbm"
+    if bound == "tensor":
+        achieved, peak, unit = dk["tflops"], peak_t, "TFLOP/s"
+        peak_kind = ("sustained" if long_region else "burst") + f" bf16 GEMM, {peaks['source']}"
+    else:
+        achieved, peak, unit = dk["gbs"], peaks["hbm"], "GB/s"
+        peak_kind = f"HBM copy, {peaks['source']}"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": _traffic(args.config, dom),
+                "kernel": dom, "kernel_ms": dk["ms_per_launch"],
+                "kernel_share_of_step": dk["share_of_step"],
+                "algorithmic_bytes": dk["bytes_per_launch"], "algorithmic_flops": dk["flops_per_launch"],
+                "peak_kind": peak_kind}
+    peak = peak_t
 
     # ---- dense comparison on the same GPU (same graph treatment)
-    dgraphs, _ = capture_steps(lambda i, ev: wl.dense_step(i), nsets, with_events=False)
+    dgraphs, _ = capture_steps(lambda i, ev: wl.dense_step(i), nsets, None)
     dense_ms = time_steps(lambda i: dgraphs[i % nsets].replay(), args.steps, args.warmup, dist_on)
     dense_ms = _max_over_ranks(dense_ms, dist_on) / args.steps
 
@@ -564,7 +696,7 @@ def main():
            "tensor_peak_frac": value / world / peak,
            "dense_ms_per_step": dense_ms, "dense_speedup": dense_ms / ms,
            "exec_gflop_per_step": wl.exec_flops / 1e9, "dense_gflop_per_step": wl.dense_flops / 1e9,
-           "roofline": roofline, "clocks": clk.summary(),
+           "roofline": roofline, "kernels": breakdown, "clocks": clk.summary(),
            "gpu_launches": int(round(launches_per_step * args.steps)),
            "launch": ("one CUDA graph per input set, replayed once per step" if args.launch == "graph"
                       else "eager calls through the Python binding"),

@@ -1,0 +1,94 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks.
+
+The path shards by tokens with no collective on the data path; the only
+cross-rank steps are the barrier and the max over ranks of the timed region.
+These tests run them on gloo (world size 2) without a GPU.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, local_ms, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        got = bench._max_over_ranks(local_ms[rank], True, device="cpu")
+        value, ms = bench.job_throughput(got, 10, world, 1e12)
+        dist.barrier()
+        q.put((rank, got, value, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, local_ms):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, local_ms, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return sorted(out)
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    out = _run(2, [12.5, 40.0])
+    for rank, got, value, ms in out:
+        assert got == 40.0  # every rank sees the slowest rank's time
+        assert ms == pytest.approx(4.0)
+        # two ranks each did 1e12 FLOP per step in 4 ms per step
+        assert value == pytest.approx(2 * 1e12 / 4e-3 / 1e12)
+
+
+def test_single_rank_passthrough():
+    import bench
+    assert bench._max_over_ranks(3.25, False) == 3.25
+    value, ms = bench.job_throughput(50.0, 5, 1, 2e9)
+    assert ms == 10.0 and value == pytest.approx(2e9 / 1e-2 / 1e12)
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0", "--ref-rows", "16"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
+
+
+def test_reference_arm_rank0_prints_one_contract_line():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--ref-rows", "16"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "config", "cpu_baseline", "e2e"):
+        assert k in d
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0

@@ -90,6 +90,41 @@ def test_c2_decode_single_type(t):
     assert err <= TOL["bf16"], err
 
 
+# Decode shapes around the tensor-core decode kernel's limits: ragged batches,
+# the largest batch it takes (256) and the first it leaves to the SIMT
+# kernels (257), K slices of 16 rows, groups of 16 rows, q up to 32.
+@pytest.mark.parametrize("law,q,B,din,dout", [
+    ("Q2xQ2", 4, 100, 768, 1536),
+    ("Q2xQ2", 4, 256, 1536, 768),
+    ("Q2xQ2", 4, 257, 768, 1536),
+    ("Q", 16, 33, 2048, 1024),
+    ("Q", 32, 17, 4096, 2048),
+    ("Q", 2, 7, 64, 128),
+    ("Q", 8, 1, 128, 512),
+    ("Q", 4, 64, 4096, 256),
+])
+def test_decode_shapes(law, q, B, din, dout):
+    err, path = run_decode(law, q, B, din, dout, "bf16", seed=B + din)
+    assert err <= TOL["bf16"], err
+    assert path == aal.AAL_PATH_DECODE
+
+
+def test_decode_negative_position_tensor_core_kernel():
+    # 64-column output groups: the tensor-core decode kernel takes this call
+    s = inputs.Stream(5)
+    x = s.normal(3, 64, 1.0, "bf16")
+    W = s.normal(64, 128, 0.125, "bf16")
+    pos = np.array([3, -1, 6], dtype=np.int64)
+    y = torch.full((3, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    aal.aal_decode_matvec("Q", 2, torch.from_numpy(pos).cuda(), x.t.cuda(), W.t.cuda(), y)
+    assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
+    got = host64(y)
+    assert np.all(np.isnan(got[1]))  # the invalid entry is skipped
+    keep = np.array([0, 2])
+    ref = oracle.decode("Q", 2, pos[keep], x.f64[keep], W.f64)
+    assert oracle.rel_err(got[keep], ref) <= TOL["bf16"]
+
+
 # -------------------------------------------------- Qwen3-8B-shaped Q_32
 def test_c3_swiglu_full_size():
     eh, ey, path = run_swiglu("Q", 32, 2048, 4096, 12288, "bf16", seq_len=2048, w_sigma_rule="D")
