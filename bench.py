@@ -42,6 +42,12 @@ L2_BYTES = 126 * 2 ** 20
 # taken with; after any change to the kernel the bench reports null.
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
+    ("c2", "gate_up"): ("579b8a67730ec9e08246ecee4d156e7f2fa801b81a81d4a4419807779dd617bd",
+                        23669760 + 1216768, "aal_tc.cu"),
+    ("c2", "down"): ("579b8a67730ec9e08246ecee4d156e7f2fa801b81a81d4a4419807779dd617bd",
+                     40182784 + 889344, "aal_tc.cu"),
+    ("c2", "decode B=64"): ("ff77e912f196505d90639f7cbc6eb5acd1b69a9b0107c7b92815250c050c401b",
+                            (2478080 + 2478080 + 2576384) // 3, "aal_decode.cu"),
 }
 
 
