@@ -86,7 +86,7 @@ def packed_positions(rows: int, seq_len: int, offset: int = 0) -> np.ndarray:
 
 # --------------------------------------------------------------------------
 # The five workloads.  Each returns a dict of Drawn tensors plus the shape
-# parameters; sizes follow the pages' shapes.
+# parameters; sizes follow the shapes of the pages' workloads.
 # --------------------------------------------------------------------------
 
 CONFIGS = {

@@ -6,7 +6,8 @@ module.  The CUDA library never calls it and shares no code with it.
 
 What it computes, and where the pages define it (all from "Change the
 Product, Keep the Parameters: Associative Algebra Layers for Transformers",
-Koziev & Oseledets, arXiv:2609.32814; page tags as in the design doc):
+Koziev & Oseledets, arXiv:2609.32814; the pages cited are the agihunt.info
+digest, the hotpaper.ai summary and the author's post on feed.hirify.me):
 
 * The multiplication table comes from a directed graph: the diagonal slots
   of a q x q block matrix are its vertices, the kept off-diagonal slots its
@@ -24,7 +25,7 @@ Koziev & Oseledets, arXiv:2609.32814; page tags as in the design doc):
   evaluates only that row of the table (agihunt.info digest, paragraph on
   mapping to the Transformer; hotpaper.ai summary, "row-typed rectangular
   projections").  The position -> type map is position mod (number of
-  groups), the plainest reading, stated in the design doc.
+  groups), the plainest reading of "absolute position".
 * Projections are Y = X W with X [tokens, din], W [din, dout] (agihunt.info
   digest, opening paragraph); din and dout are each cut into q equal groups.
 
@@ -32,7 +33,8 @@ Every function here is a plain loop over the table with a float64 matmul as
 its only library step.  Pins that tie these functions to the pages (and not
 to themselves) live in ``tests/test_oracle_pins.py``.  The SwiGLU order
 (silu(G) * U then the down projection) is a reading of the pages' "FFN
-projections" and is pinned only through its parts.
+projections" and is pinned only through its parts (SiLU at fixed points,
+the projections, and the q = 1 case against a dense SwiGLU).
 """
 from __future__ import annotations
 
