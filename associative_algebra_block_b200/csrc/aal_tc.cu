@@ -18,11 +18,12 @@
 // [M/q][q][d]; a box with extent 1 in the middle dimension pulls the rows of
 // one type class straight out of HBM.  No index buffer, no copy.
 //
-// Roles (416 threads): warps 0 and 10..12 issue TMA loads (chunk i goes to
+// Roles (448 threads): warps 0 and 10..12 issue TMA loads (chunk i goes to
 // producer warp i mod 4), warp 1 owns TMEM and issues the MMAs (one thread),
 // warps 2..9 drain TMEM to registers and write bf16 results (optionally
-// applying SiLU(g)*u or adding into the destination); two epilogue warps share
-// each 32-lane quarter of TMEM and split its columns.
+// applying SiLU(g)*u or adding into the destination; two epilogue warps share
+// each 32-lane quarter of TMEM and split its columns), and warp 13 decodes
+// the tiles into a shared-memory ring the other roles read.
 // Tiles are visited longest first: a tile's cost is the number of block
 // products in its table entry (1, 2 or 4 for the laws here, up to q for the
 // backward's diagonal blocks), and the persistent CTAs stride through the
@@ -45,7 +46,11 @@ constexpr int kEpiWarps = 8;
 // bulk-tensor copies are issued one after another at several hundred cycles
 // each whatever the box size, so consecutive K chunks go to different warps.
 constexpr int kProdWarps = 4;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 32 * (kProdWarps - 1);
+// One more warp decodes each tile once (index -> table segments and
+// coordinates) into a ring in shared memory that every role reads.
+constexpr int kSchedWarp = 2 + kEpiWarps + kProdWarps - 1;
+constexpr int kThreads = 32 * (kSchedWarp + 1);
+constexpr int kTileRing = 8;
 constexpr int kMaxPairs = 256;
 constexpr int kMaxStages = 8;
 constexpr int kSmemBudget = 224 * 1024;  // + 1 KB alignment slack, under the 227 KB per-CTA limit
@@ -499,6 +504,27 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
 
 __device__ __forceinline__ int seg_chunks(const Seg& s) { return (s.len + 63) >> 6; }
 
+// Copies the description of this role's i-th tile out of the ring and frees
+// the slot (WARP: the whole warp reads it and lane 0 arrives).
+template <bool WARP>
+__device__ __forceinline__ bool take_tile(const TileDesc* ring, uint64_t* full, uint64_t* empty,
+                                          uint32_t i, TileDesc& d, volatile int* abort) {
+  const uint32_t slot = i % kTileRing, ph = (i / kTileRing) & 1u;
+  if (WARP) {
+    if (!warp_wait(&full[slot], ph, abort)) return false;
+  } else if (!(mbar_try_wait(&full[slot], ph) || mbar_wait(&full[slot], ph, abort))) {
+    return false;
+  }
+  d = ring[slot];
+  if (WARP) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&empty[slot]);
+  } else {
+    mbar_arrive(&empty[slot]);
+  }
+  return true;
+}
+
 // --------------------------------------------------------------- the kernel
 // A_MN / B_MN: operand tiles stored MN-major (else K-major).
 // DUAL: 0 one MMA per K step; 1 two B operands (gate/up); 2 two A operands.
@@ -514,6 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ __align__(8) uint64_t done_bar;
+  __shared__ __align__(8) uint64_t tile_full[kTileRing];
+  __shared__ __align__(8) uint64_t tile_empty[kTileRing];
+  __shared__ TileDesc s_tile[kTileRing];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
@@ -524,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   const bool issuer = !PAIR || rank == 0;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int nprod = S < kProdWarps ? S : kProdWarps;  // producer warps in use
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
@@ -532,6 +562,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * kEpiWarps);
     }
     mbar_init(&done_bar, 1);
+    // a ring slot is free again once every consuming warp has copied it: the
+    // producer warps in use, the MMA thread (where this CTA issues) and the
+    // epilogue warps
+    for (int r = 0; r < kTileRing; ++r) {
+      mbar_init(&tile_full[r], 1);
+      mbar_init(&tile_empty[r], nprod + (issuer ? 1 : 0) + kEpiWarps);
+    }
     s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -555,20 +592,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   tc_fence_after();
   const uint32_t tmem = s_tmem;
 
-  if (warp == 0 || warp >= 2 + kEpiWarps) {
+  if (warp == 0 || (warp >= 2 + kEpiWarps && warp < kSchedWarp)) {
     // ------------------------------------------------------ TMA producers
     // Every producer warp walks the same chunk sequence and issues the chunks
     // i with i mod nprod == its index.  With nprod <= S a warp waiting for
     // stage i mod S to empty cannot mistake an older phase for the one it
     // needs: its previous chunk i - nprod already saw chunk i - nprod - S
     // released, and the MMAs release stages in order.
-    const int nprod = S < kProdWarps ? S : kProdWarps;
     const int pw = warp == 0 ? 0 : warp - (1 + kEpiWarps);
-    uint32_t it = 0, st = 0, ph = 0;
+    uint32_t it = 0, st = 0, ph = 0, ti = 0;
     bool ok = pw < nprod;
-    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep) {
+    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++ti) {
       TileDesc d;
-      describe(p, tile, d);
+      if (!take_tile<true>(s_tile, tile_full, tile_empty, ti, d, &s_abort)) break;
       for (int s = 0; s < d.nseg && ok; ++s) {
         const Seg sg = seg_at(d, s);
         const int nch = seg_chunks(sg);
@@ -666,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       uint64_t so = 0;  // dstage * st
       for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++tl) {
         TileDesc d;
-        describe(p, tile, d);
+        if (!take_tile<false>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
         const uint32_t buf = tl & 1u, use = tl >> 1;
         if (!(mbar_try_wait(&tempty_bar[buf], (use & 1u) ^ 1u) ||
               mbar_wait(&tempty_bar[buf], (use & 1u) ^ 1u, &s_abort))) { ok = false; break; }
@@ -743,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     const int erow = PAIR ? (int)rank * 128 : 0;  // this CTA's 128 rows of the pair's tile
     for (int tile = tile0; tile < p.ntiles; tile += tstep, ++tl) {
       TileDesc d;
-      describe(p, tile, d);
+      if (!take_tile<true>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
       d.rbase += erow;
       const uint32_t buf = tl & 1u, use = tl >> 1;
       if (!warp_wait(&tfull_bar[buf], use & 1u, &s_abort)) break;
@@ -869,6 +905,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     }
     // every TMA store of this warp must have finished before the CTA exits
     if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  } else if (warp == kSchedWarp) {
+    // ------------------------------------------------------ tile decoder
+    if (lane == 0) {
+      uint32_t i = 0;
+      for (int tile = tile0; tile < p.ntiles; tile += tstep, ++i) {
+        const uint32_t slot = i % kTileRing, ph = (i / kTileRing) & 1u;
+        if (!(mbar_try_wait(&tile_empty[slot], ph ^ 1u) ||
+              mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
+          break;
+        TileDesc d;
+        describe(p, tile, d);
+        s_tile[slot] = d;
+        mbar_arrive(&tile_full[slot]);  // release: the copy above is visible first
+      }
+    }
     __syncwarp();
   }
 
@@ -1115,12 +1167,15 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   return cuda_status(e);
 }
 
-// AAL_TC_PAIR=0 in the environment turns the CTA-pair mode off.
+// AAL_TC_PAIR=1 in the environment turns the CTA-pair mode on.  It is off by
+// default: on B200 the single-CTA kernel with four producer warps and the
+// tile decoder is as fast or faster on every shape measured (the fused
+// gate/up of the 110M FFN: 73 us single, 78 us paired).
 static bool pair_disabled() {
   static int v = -1;
   if (v < 0) {
     const char* e = getenv("AAL_TC_PAIR");
-    v = (e && e[0] == '0') ? 1 : 0;
+    v = (e && e[0] == '1') ? 0 : 1;
   }
   return v == 1;
 }

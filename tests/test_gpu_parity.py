@@ -270,3 +270,30 @@ def test_negative_decode_position_sets_device_status():
     y = torch.zeros(2, 64, dtype=torch.bfloat16, device="cuda")
     aal.aal_decode_matvec("Q", 2, torch.tensor([3, -1], device="cuda"), x, W, y)
     assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
+
+
+# ------------------------------------------------------ CTA-pair tcgen05 mode
+_PAIR_CHILD = r"""
+import sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
+from gpu_cases import TOL, run_swiglu, run_project
+import associative_algebra_block_b200 as aal
+eh, ey, path = run_swiglu('Q2xQ2', 4, 3072, 768, 1536, 'bf16', seq_len=1536)
+assert path == aal.AAL_PATH_TENSOR, path
+assert eh <= TOL['bf16'] and ey <= TOL['bf16'], (eh, ey)
+e, path = run_project('Q', 4, 2048, 512, 1024, 'bf16', seq_len=1024)
+assert e <= TOL['bf16'], e
+print('ok')
+"""
+
+
+@pytest.mark.gpu
+def test_cta_pair_mode_parity():
+    # the pair mode is chosen once per process from the environment
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _PAIR_CHILD, root], capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, AAL_TC_PAIR="1"))
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
