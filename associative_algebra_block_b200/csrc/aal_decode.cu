@@ -662,6 +662,10 @@ constexpr int kMmaKc = 192;       // weight rows staged per round
 constexpr int kMmaWStride = 72;   // staged weight row: 64 columns + 8 pad (144 bytes)
 constexpr int kMmaPStride = 68;   // fp32 partial row: 64 columns + 4 pad
 
+// Shared memory of the staging area (weight rows + activations), 16-byte multiple.
+__host__ __device__ inline size_t mma_stage_bytes(int Bp) {
+  return (size_t)kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
+}
 __device__ __forceinline__ uint32_t dec_smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
@@ -690,11 +694,14 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, cons
 
 // NT: n-tiles (8 entries) per warp; warps 0..3 take the four 16-column
 // m-tiles, warps 4..7 the same m-tiles for the odd n-tiles.
-// Latency is the cost at these sizes, so the first round's copies start
-// before the row types are known: the weight rows of the whole round are
-// fetched (later rounds fetch only the groups some entry uses), the
-// activations unmasked, and an entry's table row is applied to its operand
-// fragment in registers.
+// Latency is the cost at these sizes, so: each thread's position load is in
+// flight while the first round's copies are issued (all weight rows of the
+// round, the activations unmasked; later rounds fetch only the groups some
+// entry uses); an entry's table row is applied to its operand fragment in
+// registers; and the split-K partials are pushed into the owning CTA's
+// shared memory, so one cluster barrier (whose arrival half is posted at the
+// start) separates the MMAs from the sums and no CTA reads a peer afterwards.
+// Entry n is owned (summed and written) by CTA n mod cl of the cluster.
 template <int NT>
 __global__ void __launch_bounds__(256)
 k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
@@ -703,9 +710,11 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
              long long ldy, int bi, int bo, int slice) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ int s_type[kMmaMaxB];
-  __shared__ unsigned long long s_present;
+  __shared__ unsigned s_pres[8][2];
   __shared__ unsigned char s_used[64];  // groups of the CTA's K slice that some entry uses
   cg::cluster_group cluster = cg::this_cluster();
+  // every CTA of the cluster is running before any writes into a peer
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c0 = blockIdx.x * kMmaCols;
@@ -713,11 +722,18 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   const int ks0 = blockIdx.z * slice;  // first weight row of this CTA
   const int Bp = (B + 7) & ~7;
   const int ntiles = Bp >> 3;
-  const int xs_stride = kMmaKc + 8;  // staged activation row, bf16
+  const int cl = (int)gridDim.z;
+  const int rows_own = (Bp + cl - 1) / cl;  // entries owned per CTA (upper bound)
+  const int xs_stride = kMmaKc + 8;         // staged activation row, bf16
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(dsm);
   __nv_bfloat16* Xs = Ws + kMmaKc * kMmaWStride;
-  float* P = reinterpret_cast<float*>(dsm);  // reused after the MMAs
+  // receive area: [source rank][owned entry][64 columns] fp32, after staging
+  float* R = reinterpret_cast<float*>(dsm + mma_stage_bytes(Bp));
   const int g0 = ks0 / bi, ng = (ks0 + slice - 1) / bi - g0 + 1;
+
+  // the position of entry tid is in flight while the copies are issued
+  long long my_pos = -1;
+  if (tid < B) my_pos = pos[tid];
 
   auto stage = [&](int r0, int rows, bool all_rows) {
     for (int i = tid; i < rows * 8; i += blockDim.x) {
@@ -726,9 +742,11 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
         cp_async16(dec_smem_u32(Ws + r * kMmaWStride + ch * 8),
                    W + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
     }
-    const int xch = rows >> 3;
-    for (int i = tid; i < Bp * xch; i += blockDim.x) {
-      const int n = i / xch, ch = i - n * xch;
+    // item i = n * xch + ch, walked without a division per item
+    const int xch = rows >> 3, dq = 256 / xch, dr = 256 - dq * xch;
+    int n = tid / xch, ch = tid - n * xch;
+    for (; n < Bp; n += dq, ch += dr) {
+      if (ch >= xch) { ch -= xch; ++n; if (n >= Bp) break; }
       const bool in = n < B;
       cp_async16(dec_smem_u32(Xs + n * xs_stride + ch * 8),
                  in ? x + (long long)n * ldx + r0 + ch * 8 : x, in ? 16u : 0u);
@@ -739,30 +757,31 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   // round 0's copies go out first
   stage(ks0, min(kMmaKc, slice), true);
 
-  // 1. row type of every entry; -1 for padding and invalid positions
-  if (tid == 0) s_present = 0ull;
-  __syncthreads();
-  for (int b = tid; b < Bp; b += blockDim.x) {
-    int t = -1;
-    if (b < B) {
-      const long long p = pos[b];
-      if (p < 0) {
-        if (blockIdx.x == 0 && blockIdx.z == 0) flag_device_error(kDevBounds);
-      } else {
-        t = (int)(p % q);
-        atomicOr(&s_present, 1ull << t);
-      }
+  // 1. row type of every entry (-1 for padding and invalid positions) and
+  //    the set of types present
+  int t = -1;
+  if (tid < B) {
+    if (my_pos < 0) {
+      if (blockIdx.x == 0 && blockIdx.z == 0) flag_device_error(kDevBounds);
+    } else {
+      t = (int)(my_pos % q);
     }
-    s_type[b] = t;
   }
+  if (tid < Bp) s_type[tid] = t;
+  const unsigned lo = __reduce_or_sync(0xffffffffu, (t >= 0 && t < 32) ? 1u << t : 0u);
+  const unsigned hi = __reduce_or_sync(0xffffffffu, t >= 32 ? 1u << (t - 32) : 0u);
+  if (lane == 0) { s_pres[warp][0] = lo; s_pres[warp][1] = hi; }
   __syncthreads();
   // 2. which groups a of the slice some present type uses with output group k
   if (tid < ng) {
+    unsigned long long pres = 0ull;
+#pragma unroll
+    for (int w = 0; w < 8; ++w)
+      pres |= (unsigned long long)s_pres[w][0] | ((unsigned long long)s_pres[w][1] << 32);
     const int a = g0 + tid;
-    const unsigned long long pres = s_present;
     bool u = false;
-    for (int t = 0; t < q && !u; ++t)
-      if ((pres >> t) & 1ull) u = in_table(law, t, k, a);
+    for (int tt = 0; tt < q && !u; ++tt)
+      if ((pres >> tt) & 1ull) u = in_table(law, tt, k, a);
     s_used[tid] = u ? 1 : 0;
   }
 
@@ -773,8 +792,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
     for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
   const int mt = warp & 3, nt0 = warp >> 2;
   const int g = lane >> 2;
-  // row types of the entries whose B fragments this thread holds
-  int my_t[NT];
+  int my_t[NT];  // row types of the entries whose B fragments this thread holds
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     const int n = (nt0 + 2 * j) * 8 + g;
@@ -789,80 +807,87 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
     __syncthreads();
     // 3. MMAs over the used 16-row steps; an entry whose table row does not
     //    use the step's group contributes zeros
-    int a_prev = -1;
+    int a = r0 / bi, a_end = (a + 1) * bi - r0;  // group of step kk, and where it ends
+    bool used = s_used[a - g0];
     unsigned keep = 0;  // bit j: entry of n-tile j uses group a
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+      if (my_t[j] >= 0 && in_table(law, my_t[j], k, a)) keep |= 1u << j;
+#pragma unroll 2
     for (int kk = 0; kk < rows; kk += 16) {
-      const int a = (r0 + kk) / bi;
-      if (!s_used[a - g0]) continue;
-      if (a != a_prev) {
+      if (kk >= a_end) {
+        ++a;
+        a_end += bi;
+        used = s_used[a - g0];
         keep = 0;
 #pragma unroll
         for (int j = 0; j < NT; ++j)
           if (my_t[j] >= 0 && in_table(law, my_t[j], k, a)) keep |= 1u << j;
-        a_prev = a;
       }
+      if (!used) continue;
       uint32_t af[4];
       const int arow = kk + (lane & 7) + ((lane >> 4) << 3);
       const int acol = mt * 16 + (((lane >> 3) & 1) << 3);
       ldsm_x4_trans(dec_smem_u32(Ws + arow * kMmaWStride + acol), af);
+      uint32_t bf[NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         const int nt = nt0 + 2 * j;
         if (nt < ntiles) {
-          uint32_t bf[2];
           const int brow = nt * 8 + (lane & 7);
           const int bcol = kk + (((lane >> 3) & 1) << 3);
-          ldsm_x2(dec_smem_u32(Xs + brow * xs_stride + bcol), bf);
-          if (!((keep >> j) & 1u)) { bf[0] = 0u; bf[1] = 0u; }
-          mma_bf16_16816(acc[j], af, bf);
+          ldsm_x2(dec_smem_u32(Xs + brow * xs_stride + bcol), bf[j]);
+          if (!((keep >> j) & 1u)) { bf[j][0] = 0u; bf[j][1] = 0u; }
         }
       }
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+        if (nt0 + 2 * j < ntiles) mma_bf16_16816(acc[j], af, bf[j]);
     }
-    __syncthreads();
+    if (kc + kMmaKc < slice) __syncthreads();  // staging is refilled next round
   }
-  // 4. fp32 partials [entry][column] in shared memory
+  // 4. push the fp32 partials to their owners: entry n -> CTA n mod cl,
+  //    slot [this rank][n / cl]
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   const int c = lane & 3;
+  const unsigned my_rank = cluster.block_rank();
+  const int rstride = rows_own * kMmaPStride;  // floats per source rank
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     const int nt = nt0 + 2 * j;
     if (nt < ntiles) {
-      const int n = nt * 8 + 2 * c, m = mt * 16 + g;
-      P[n * kMmaPStride + m] = acc[j][0];
-      P[(n + 1) * kMmaPStride + m] = acc[j][1];
-      P[n * kMmaPStride + m + 8] = acc[j][2];
-      P[(n + 1) * kMmaPStride + m + 8] = acc[j][3];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = nt * 8 + 2 * c + e;
+        float* dst = cluster.map_shared_rank(R, n % cl) + my_rank * rstride + (n / cl) * kMmaPStride;
+        const int m = mt * 16 + g;
+        dst[m] = acc[j][e];
+        dst[m + 8] = acc[j][2 + e];
+      }
     }
   }
-  cluster.sync();
-  // 5. CTA z sums rows z, z + cl, ... over the cluster (4 columns per thread,
-  //    every peer's load in flight at once) and writes them
-  const int cl = (int)gridDim.z, z = (int)blockIdx.z;
-  const int my_rows = (Bp - z + cl - 1) / cl;
-  for (int i = tid; i < my_rows * 16; i += blockDim.x) {
-    const int n = z + cl * (i >> 4), ch = i & 15;
+  cluster.sync();  // every partial has landed in its owner
+  // 5. owners sum their entries over the cluster's ranks and write them
+  for (int i = tid; i < rows_own * 16; i += blockDim.x) {
+    const int jr = i >> 4, ch = i & 15;
+    const int n = (int)my_rank + cl * jr;
     if (n >= B || s_type[n] < 0) continue;
-    float4 u[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < cl)
-        u[r] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(P, r) + n * kMmaPStride + ch * 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < cl) { v.x += u[r].x; v.y += u[r].y; v.z += u[r].z; v.w += u[r].w; }
+    for (int r = 0; r < cl; ++r) {
+      const float4 u = *reinterpret_cast<const float4*>(R + r * rstride + jr * kMmaPStride + ch * 4);
+      v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+    }
     uint2 o;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
     h[0] = __floats2bfloat162_rn(v.x, v.y);
     h[1] = __floats2bfloat162_rn(v.z, v.w);
     *reinterpret_cast<uint2*>(y + (long long)n * ldy + c0 + ch * 4) = o;
   }
-  cluster.sync();  // no CTA leaves while a peer still reads its partials
 }
 
-static size_t mma_smem_bytes(int Bp) {
-  const size_t stage = (size_t)kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
-  const size_t part = (size_t)Bp * kMmaPStride * 4;
-  return stage > part ? stage : part;
+static size_t mma_smem_bytes(int Bp, int cl) {
+  const size_t recv = (size_t)cl * ((Bp + cl - 1) / cl) * kMmaPStride * 4;
+  return mma_stage_bytes(Bp) + recv;
 }
 
 template <int NT>
@@ -870,7 +895,7 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
                               const aal_mat& x, const aal_mat& W, const aal_mat& y, int bi, int bo,
                               long long dout, cudaStream_t s) {
   const int Bp = (B + 7) & ~7;
-  const size_t smem = mma_smem_bytes(Bp);
+  const size_t smem = mma_smem_bytes(Bp, cl);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -878,7 +903,7 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_done & bit)) {
     e = cudaFuncSetAttribute(k_decode_mma<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)mma_smem_bytes(kMmaMaxB));
+                             (int)mma_smem_bytes(kMmaMaxB, 8));
     if (e != cudaSuccess) return e;
     attr_done |= bit;
   }
