@@ -36,18 +36,19 @@ from associative_algebra_block_b200 import inputs  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu
-# capture of this command on a B200 (summaries under profiles/).  A figure is
-# used only while the tensor-core source still hashes to the value it was
-# taken with; after any change to the kernel the bench reports null.
+# DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
+# ``python bench.py --steps 3 --warmup 3 --no-cpu-baseline`` on a B200
+# (summaries under profiles/).  A figure is used only while the kernel's source
+# file still hashes to the value it was taken with; after any change to the
+# kernel the bench reports null.
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
-    ("c2", "gate_up"): ("579b8a67730ec9e08246ecee4d156e7f2fa801b81a81d4a4419807779dd617bd",
-                        23669760 + 1216768, "aal_tc.cu"),
-    ("c2", "down"): ("579b8a67730ec9e08246ecee4d156e7f2fa801b81a81d4a4419807779dd617bd",
-                     40182784 + 889344, "aal_tc.cu"),
-    ("c2", "decode B=64"): ("ff77e912f196505d90639f7cbc6eb5acd1b69a9b0107c7b92815250c050c401b",
-                            (2478080 + 2478080 + 2576384) // 3, "aal_decode.cu"),
+    ("c2", "gate_up"): ("7b4dbbdd970c1f53d959e716da9b8e65cce5c962aa7fc6f0820cdda6ddad05b2",
+                        23669504 + 1120256, "aal_tc.cu"),
+    ("c2", "down"): ("7b4dbbdd970c1f53d959e716da9b8e65cce5c962aa7fc6f0820cdda6ddad05b2",
+                     40178176 + 857856, "aal_tc.cu"),
+    ("c2", "decode B=64"): ("4399e2d996d5b6224b7d7aea0abb3dd46e5543be0d7e4eeb39dd6b8824032fc0",
+                            (2488064 + 2487808 + 2586112) // 3, "aal_decode.cu"),
 }
 
 
