@@ -35,11 +35,12 @@ AAL_TYPES_POSITION, AAL_TYPES_EXPLICIT = 0, 1
 AAL_PATH_AUTO, AAL_PATH_TENSOR, AAL_PATH_GENERAL, AAL_PATH_DECODE = 0, 1, 2, 3
 
 EXPORTS = ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd", "aal_decode_matvec",
-           "aal_square_product", "aal_block_table", "aal_block_product_count",
+           "aal_swiglu_decode", "aal_square_product", "aal_block_table", "aal_block_product_count",
            "aal_get_device_status", "aal_status_string", "aal_set_path_policy",
            "aal_last_path", "aal_launch_count", "aal_version", "aal_set_timing_events")
 AAL_KERNEL_PROJECT, AAL_KERNEL_GATE_UP, AAL_KERNEL_BWD_DX = 1, 2, 3
 AAL_KERNEL_BWD_DW, AAL_KERNEL_SQUARE, AAL_KERNEL_DECODE = 4, 5, 6
+AAL_KERNEL_DECODE_GATE_UP = 7
 
 
 class AalError(RuntimeError):
@@ -77,6 +78,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
             "aal_project_fwd": ([i32, i32, AalRowTypeRule, AalMat, AalMat, AalMat, vp], i32),
             "aal_swiglu_fwd": ([i32, i32, AalRowTypeRule, AalMat, AalMat, AalMat, AalMat, AalMat,
                                 AalMat, vp], i32),
+            "aal_swiglu_decode": ([i32, i32, vp, AalMat, AalMat, AalMat, AalMat, AalMat, AalMat, vp],
+                                  i32),
             "aal_project_bwd": ([i32, i32, AalRowTypeRule, AalMat, AalMat, AalMat, AalMat, AalMat,
                                  i32, vp], i32),
             "aal_decode_matvec": ([i32, i32, vp, AalMat, AalMat, AalMat, vp], i32),
@@ -183,6 +186,14 @@ def aal_decode_matvec(law, q, positions, x, W, y, stream=None):
         raise ValueError("positions must be int64")
     _check(load().aal_decode_matvec(_law(law), q, positions.data_ptr() if positions.numel() else None,
                                     mat(x), mat(W), mat(y), _stream(stream)), "aal_decode_matvec")
+
+
+def aal_swiglu_decode(law, q, positions, x, Wg, Wu, Wd, h, y, stream=None):
+    if positions.dtype != torch.int64:
+        raise ValueError("positions must be int64")
+    _check(load().aal_swiglu_decode(_law(law), q, positions.data_ptr() if positions.numel() else None,
+                                    mat(x), mat(Wg), mat(Wu), mat(Wd), mat(h), mat(y), _stream(stream)),
+           "aal_swiglu_decode")
 
 
 def aal_square_product(law, q, X, W, Z, stream=None):

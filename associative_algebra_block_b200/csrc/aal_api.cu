@@ -209,6 +209,60 @@ aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* positions, a
   return st;
 }
 
+aal_status aal_swiglu_decode(int32_t law, int32_t q, const int64_t* positions, aal_mat x,
+                             aal_mat Wg, aal_mat Wu, aal_mat Wd, aal_mat h, aal_mat y, void* stream) {
+  if (!valid_law(law, q) || !valid_mat(x) || !valid_mat(Wg) || !valid_mat(Wu) || !valid_mat(Wd) ||
+      !valid_mat(h) || !valid_mat(y))
+    return AAL_ERR_INVALID_ARG;
+  if (x.dtype != Wg.dtype || x.dtype != Wu.dtype || x.dtype != Wd.dtype || x.dtype != h.dtype ||
+      x.dtype != y.dtype)
+    return AAL_ERR_UNSUPPORTED;
+  const long long B = x.rows, D = x.cols, F = Wg.cols;
+  if (Wg.rows != D || Wu.rows != D || Wu.cols != F || Wd.rows != F || Wd.cols != D ||
+      h.rows != B || h.cols != F || y.rows != B || y.cols != D)
+    return AAL_ERR_INVALID_ARG;
+  if (D % q || F % q) return AAL_ERR_INVALID_ARG;
+  if (B > 0 && positions == nullptr) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (B == 0 || D == 0 || F == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  int path = AAL_PATH_DECODE;
+  aal_status st = AAL_OK;
+  bool handled = false;
+  if (t_policy != AAL_PATH_GENERAL) {
+    st = timed(AAL_KERNEL_DECODE_GATE_UP, s, [&] {
+      return decode_gate_up(law, q, positions, x, Wg, Wu, h, s, &handled);
+    });
+    if (st != AAL_OK) return st;
+    if (!handled && t_policy == AAL_PATH_TENSOR) return AAL_ERR_UNSUPPORTED;
+  }
+  RowTypes rt;
+  rt.kind = kTypesPositions64;
+  rt.q = q;
+  rt.seq_len = 1;
+  rt.pos_offset = 0;
+  rt.types = nullptr;
+  rt.positions = positions;
+  if (!handled) {
+    st = timed(AAL_KERNEL_DECODE_GATE_UP, s, [&] { return simt_swiglu_gate_up(law, q, rt, x, Wg, Wu, h, s); });
+    if (st != AAL_OK) return st;
+    path = AAL_PATH_GENERAL;
+  }
+  handled = false;
+  if (t_policy != AAL_PATH_GENERAL) {
+    st = timed(AAL_KERNEL_DECODE, s, [&] { return decode_matvec(law, q, positions, h, Wd, y, s, &handled); });
+    if (st != AAL_OK) return st;
+  }
+  if (!handled) {
+    if (t_policy == AAL_PATH_TENSOR) return AAL_ERR_UNSUPPORTED;
+    st = simt_project(law, q, rt, h, Wd, y, s);
+    if (st != AAL_OK) return st;
+    path = AAL_PATH_GENERAL;
+  }
+  note_path(path);
+  return AAL_OK;
+}
+
 aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat W, aal_mat Z,
                               void* stream) {
   if (!valid_law(law, q) || !valid_mat(X) || !valid_mat(W) || !valid_mat(Z))
@@ -276,7 +330,7 @@ const char* aal_status_string(int32_t status) {
 }
 
 aal_status aal_set_timing_events(int32_t kernel, void* before, void* after) {
-  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_DECODE) return AAL_ERR_INVALID_ARG;
+  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_DECODE_GATE_UP) return AAL_ERR_INVALID_ARG;
   t_ev_before[kernel] = (cudaEvent_t)before;
   t_ev_after[kernel] = (cudaEvent_t)after;
   return AAL_OK;

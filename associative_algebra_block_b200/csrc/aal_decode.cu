@@ -658,13 +658,14 @@ static cudaError_t launch_typed(int law, int q, const int64_t* positions, int B,
 // (B = X^T, rows of X), K the weight rows.
 constexpr int kMmaCols = 64;      // output columns per CTA
 constexpr int kMmaMaxB = 256;     // batch entries per launch
+constexpr int kMmaMaxBGU = 128;   // batch entries per launch of the fused gate/up kernel
 constexpr int kMmaKc = 192;       // weight rows staged per round
 constexpr int kMmaWStride = 72;   // staged weight row: 64 columns + 8 pad (144 bytes)
 constexpr int kMmaPStride = 68;   // fp32 partial row: 64 columns + 4 pad
 
 // Shared memory of the staging area (weight rows + activations), 16-byte multiple.
-__host__ __device__ inline size_t mma_stage_bytes(int Bp) {
-  return (size_t)kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
+__host__ __device__ inline size_t mma_stage_bytes(int Bp, int nw) {
+  return (size_t)nw * kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
 }
 __device__ __forceinline__ uint32_t dec_smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -702,11 +703,16 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, cons
 // shared memory, so one cluster barrier (whose arrival half is posted at the
 // start) separates the MMAs from the sums and no CTA reads a peer afterwards.
 // Entry n is owned (summed and written) by CTA n mod cl of the cluster.
-template <int NT>
+// GU: the gate/up pair of a SwiGLU FFN in one launch: W is Wg and W2 is Wu
+// (same shape and stride), both read against the same staged activations, and
+// the owner writes y = silu(x Wg) * (x Wu) (agihunt.info digest, SwiGLU
+// figures; the activation is applied to the fp32 sums, rounded once to bf16).
+template <int NT, bool GU>
 __global__ void __launch_bounds__(256)
 k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
              const __nv_bfloat16* __restrict__ x, long long ldx,
-             const __nv_bfloat16* __restrict__ W, long long ldw, __nv_bfloat16* __restrict__ y,
+             const __nv_bfloat16* __restrict__ W, const __nv_bfloat16* __restrict__ W2,
+             long long ldw, __nv_bfloat16* __restrict__ y,
              long long ldy, int bi, int bo, int slice) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ int s_type[kMmaMaxB];
@@ -725,10 +731,11 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   const int cl = (int)gridDim.z;
   const int rows_own = (Bp + cl - 1) / cl;  // entries owned per CTA (upper bound)
   const int xs_stride = kMmaKc + 8;         // staged activation row, bf16
+  constexpr int NW = GU ? 2 : 1;  // weight tiles staged per round
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(dsm);
-  __nv_bfloat16* Xs = Ws + kMmaKc * kMmaWStride;
-  // receive area: [source rank][owned entry][64 columns] fp32, after staging
-  float* R = reinterpret_cast<float*>(dsm + mma_stage_bytes(Bp));
+  __nv_bfloat16* Xs = Ws + NW * kMmaKc * kMmaWStride;
+  // receive area: [operand][source rank][owned entry][64 columns] fp32, after staging
+  float* R = reinterpret_cast<float*>(dsm + mma_stage_bytes(Bp, NW));
   const int g0 = ks0 / bi, ng = (ks0 + slice - 1) / bi - g0 + 1;
 
   // the position of entry tid is in flight while the copies are issued
@@ -738,9 +745,13 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   auto stage = [&](int r0, int rows, bool all_rows) {
     for (int i = tid; i < rows * 8; i += blockDim.x) {
       const int r = i >> 3, ch = i & 7;
-      if (all_rows || s_used[(r0 + r) / bi - g0])
+      if (all_rows || s_used[(r0 + r) / bi - g0]) {
         cp_async16(dec_smem_u32(Ws + r * kMmaWStride + ch * 8),
                    W + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
+        if (GU)
+          cp_async16(dec_smem_u32(Ws + (kMmaKc + r) * kMmaWStride + ch * 8),
+                     W2 + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
+      }
     }
     // item i = n * xch + ch, walked without a division per item
     const int xch = rows >> 3, dq = 256 / xch, dr = 256 - dq * xch;
@@ -785,11 +796,13 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
     s_used[tid] = u ? 1 : 0;
   }
 
-  float acc[NT][4];
+  float acc[NW][NT][4];
 #pragma unroll
-  for (int j = 0; j < NT; ++j)
+  for (int o = 0; o < NW; ++o)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[o][j][e] = 0.f;
   const int mt = warp & 3, nt0 = warp >> 2;
   const int g = lane >> 2;
   int my_t[NT];  // row types of the entries whose B fragments this thread holds
@@ -825,10 +838,12 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
           if (my_t[j] >= 0 && in_table(law, my_t[j], k, a)) keep |= 1u << j;
       }
       if (!used) continue;
-      uint32_t af[4];
+      uint32_t af[NW][4];
       const int arow = kk + (lane & 7) + ((lane >> 4) << 3);
       const int acol = mt * 16 + (((lane >> 3) & 1) << 3);
-      ldsm_x4_trans(dec_smem_u32(Ws + arow * kMmaWStride + acol), af);
+#pragma unroll
+      for (int o = 0; o < NW; ++o)
+        ldsm_x4_trans(dec_smem_u32(Ws + (o * kMmaKc + arow) * kMmaWStride + acol), af[o]);
       uint32_t bf[NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -842,7 +857,10 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
       }
 #pragma unroll
       for (int j = 0; j < NT; ++j)
-        if (nt0 + 2 * j < ntiles) mma_bf16_16816(acc[j], af, bf[j]);
+        if (nt0 + 2 * j < ntiles) {
+#pragma unroll
+          for (int o = 0; o < NW; ++o) mma_bf16_16816(acc[o][j], af[o], bf[j]);
+        }
     }
     if (kc + kMmaKc < slice) __syncthreads();  // staging is refilled next round
   }
@@ -852,6 +870,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   const int c = lane & 3;
   const unsigned my_rank = cluster.block_rank();
   const int rstride = rows_own * kMmaPStride;  // floats per source rank
+  const int ostride = cl * rstride;             // floats per operand
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
     const int nt = nt0 + 2 * j;
@@ -861,8 +880,11 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
         const int n = nt * 8 + 2 * c + e;
         float* dst = cluster.map_shared_rank(R, n % cl) + my_rank * rstride + (n / cl) * kMmaPStride;
         const int m = mt * 16 + g;
-        dst[m] = acc[j][e];
-        dst[m + 8] = acc[j][2 + e];
+#pragma unroll
+        for (int o = 0; o < NW; ++o) {
+          dst[o * ostride + m] = acc[o][j][e];
+          dst[o * ostride + m + 8] = acc[o][j][2 + e];
+        }
       }
     }
   }
@@ -877,6 +899,18 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
       const float4 u = *reinterpret_cast<const float4*>(R + r * rstride + jr * kMmaPStride + ch * 4);
       v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
     }
+    if (GU) {
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < cl; ++r) {
+        const float4 u = *reinterpret_cast<const float4*>(R + ostride + r * rstride + jr * kMmaPStride + ch * 4);
+        w.x += u.x; w.y += u.y; w.z += u.z; w.w += u.w;
+      }
+      // silu(g) * u = g / (1 + e^-g) * u
+      v.x = __fdividef(v.x, 1.0f + __expf(-v.x)) * w.x;
+      v.y = __fdividef(v.y, 1.0f + __expf(-v.y)) * w.y;
+      v.z = __fdividef(v.z, 1.0f + __expf(-v.z)) * w.z;
+      v.w = __fdividef(v.w, 1.0f + __expf(-v.w)) * w.w;
+    }
     uint2 o;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
     h[0] = __floats2bfloat162_rn(v.x, v.y);
@@ -885,25 +919,26 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   }
 }
 
-static size_t mma_smem_bytes(int Bp, int cl) {
-  const size_t recv = (size_t)cl * ((Bp + cl - 1) / cl) * kMmaPStride * 4;
-  return mma_stage_bytes(Bp) + recv;
+static size_t mma_smem_bytes(int Bp, int cl, int nw) {
+  const size_t recv = (size_t)nw * cl * ((Bp + cl - 1) / cl) * kMmaPStride * 4;
+  return mma_stage_bytes(Bp, nw) + recv;
 }
 
-template <int NT>
+template <int NT, bool GU>
 static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, int B,
-                              const aal_mat& x, const aal_mat& W, const aal_mat& y, int bi, int bo,
-                              long long dout, cudaStream_t s) {
+                              const aal_mat& x, const aal_mat& W, const aal_mat* W2, const aal_mat& y,
+                              int bi, int bo, long long dout, cudaStream_t s) {
+  constexpr int NW = GU ? 2 : 1;
   const int Bp = (B + 7) & ~7;
-  const size_t smem = mma_smem_bytes(Bp, cl);
+  const size_t smem = mma_smem_bytes(Bp, cl, NW);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static unsigned long long attr_done = 0;  // per device (bit dev % 64)
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_done & bit)) {
-    e = cudaFuncSetAttribute(k_decode_mma<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)mma_smem_bytes(kMmaMaxB, 8));
+    e = cudaFuncSetAttribute(k_decode_mma<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)mma_smem_bytes(GU ? kMmaMaxBGU : kMmaMaxB, 8, NW));
     if (e != cudaSuccess) return e;
     attr_done |= bit;
   }
@@ -919,8 +954,9 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
   attr[0].val.clusterDim.z = cl;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_mma<NT>, law, q, positions, B,
-                            (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr, W.ld,
+  return cudaLaunchKernelEx(&cfg, k_decode_mma<NT, GU>, law, q, positions, B,
+                            (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr,
+                            (const __nv_bfloat16*)(GU ? W2->ptr : W.ptr), W.ld,
                             (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)(x.cols / cl));
 }
 
@@ -948,6 +984,40 @@ static bool typed_disabled() {
   return v == 1;
 }
 
+// Gate and up projections of a SwiGLU FFN for a decode batch in one launch,
+// h = silu(x Wg) * (x Wu); batches above 128 entries go in chunks of 128.
+aal_status decode_gate_up(int law, int q, const int64_t* positions, const aal_mat& x,
+                          const aal_mat& Wg, const aal_mat& Wu, const aal_mat& h, cudaStream_t s,
+                          bool* handled) {
+  *handled = false;
+  const long long B = x.rows, dout = Wg.cols;
+  if (B == 0 || dout == 0) { *handled = true; return AAL_OK; }
+  const int bi = (int)(x.cols / q), bo = (int)(dout / q);
+  if (!(x.dtype == AAL_BF16 && Wg.dtype == AAL_BF16 && Wu.dtype == AAL_BF16 && h.dtype == AAL_BF16 &&
+        q <= 64 && bo % kMmaCols == 0 && bi % 16 == 0 && aligned16(x) && aligned16(Wg) &&
+        aligned16(Wu) && Wg.ld == Wu.ld && aligned16(h) && x.cols <= INT_MAX && dout <= INT_MAX &&
+        !mma_disabled()))
+    return AAL_OK;
+  *handled = true;
+  int cl = 8;
+  while (cl > 1 && (x.cols % (16 * cl)) != 0) cl >>= 1;
+  for (long long b0 = 0; b0 < B; b0 += kMmaMaxBGU) {
+    const int nb = (int)(B - b0 < kMmaMaxBGU ? B - b0 : kMmaMaxBGU);
+    aal_mat xs = x, hs = h;
+    xs.ptr = (char*)x.ptr + (size_t)b0 * x.ld * 2;
+    xs.rows = nb;
+    hs.ptr = (char*)h.ptr + (size_t)b0 * h.ld * 2;
+    hs.rows = nb;
+    cudaError_t e;
+    if (nb <= 16) e = launch_mma<1, true>(cl, law, q, positions + b0, nb, xs, Wg, &Wu, hs, bi, bo, dout, s);
+    else if (nb <= 64) e = launch_mma<4, true>(cl, law, q, positions + b0, nb, xs, Wg, &Wu, hs, bi, bo, dout, s);
+    else e = launch_mma<8, true>(cl, law, q, positions + b0, nb, xs, Wg, &Wu, hs, bi, bo, dout, s);
+    note_launch();
+    if (e != cudaSuccess) return AAL_ERR_CUDA;
+  }
+  return AAL_OK;
+}
+
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
                          const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled) {
   *handled = true;
@@ -965,9 +1035,9 @@ aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat
     int cl = 8;
     while (cl > 1 && (x.cols % (16 * cl)) != 0) cl >>= 1;
     cudaError_t e;
-    if (B <= 16) e = launch_mma<1>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
-    else if (B <= 64) e = launch_mma<4>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
-    else e = launch_mma<16>(cl, law, q, positions, (int)B, x, W, y, bi, bo, dout, s);
+    if (B <= 16) e = launch_mma<1, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
+    else if (B <= 64) e = launch_mma<4, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
+    else e = launch_mma<16, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
     note_launch();
     return cuda_status(e);
   }

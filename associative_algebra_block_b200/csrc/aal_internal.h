@@ -87,6 +87,9 @@ aal_status simt_square(int law, int q, const aal_mat& X, const aal_mat& W, const
                        cudaStream_t s);
 
 // ----------------------------------------------------------------- decode path
+aal_status decode_gate_up(int law, int q, const int64_t* positions, const aal_mat& x,
+                          const aal_mat& Wg, const aal_mat& Wu, const aal_mat& h, cudaStream_t s,
+                          bool* handled);
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
                          const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled);
 

@@ -47,8 +47,6 @@ NCU_TRAFFIC = {
                         23669504 + 1120256, "aal_tc.cu"),
     ("c2", "down"): ("7b4dbbdd970c1f53d959e716da9b8e65cce5c962aa7fc6f0820cdda6ddad05b2",
                      40178176 + 857856, "aal_tc.cu"),
-    ("c2", "decode B=64"): ("4399e2d996d5b6224b7d7aea0abb3dd46e5543be0d7e4eeb39dd6b8824032fc0",
-                            (2488064 + 2487808 + 2586112) // 3, "aal_decode.cu"),
 }
 
 
@@ -93,7 +91,7 @@ def _exec_flops_proj(law, q, M, din, dout):
 
 
 class SwigluDecode:
-    """Algebraic SwiGLU forward over M packed tokens + decode matvecs."""
+    """Algebraic SwiGLU forward over M packed tokens + FFN decode steps."""
 
     def __init__(self, name, law, q, M, D, F, seq_len, w_sigma_rule="din", decode_batches=(1, 8, 64)):
         self.name, self.law, self.q, self.M, self.D, self.F = name, law, q, M, D, F
@@ -110,7 +108,8 @@ class SwigluDecode:
     def config(self):
         return {"workload": f"{self.name}: {self.law} q={self.q} SwiGLU FFN fwd d={self.D} "
                             f"ffn={self.F} M={self.M} ({self.M // self.seq_len}x{self.seq_len} tokens) "
-                            f"+ decode matvec B={'/'.join(map(str, self.decode_batches))}",
+                            f"+ FFN decode matvecs B={'/'.join(map(str, self.decode_batches))} "
+                            f"(gate/up/SiLU*mul in one launch, then down)",
                 "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F,
                 "seq_len": self.seq_len, "decode_batches": list(self.decode_batches)}
 
@@ -133,11 +132,9 @@ class SwigluDecode:
             st = inputs.Stream(seed + 100 + i)
             for B in self.decode_batches:
                 x = st.normal(B, self.D, 1.0, "bf16", want_f64=False).t.cuda()
-                h = st.normal(B, self.F, 1.0, "bf16", want_f64=False).t.cuda()
                 pos = torch.from_numpy(st.positions(B, self.seq_len)).cuda()
-                s["dec"].append(dict(x=x, h=h, pos=pos,
-                                     g=torch.empty(B, self.F, dtype=torch.bfloat16, device="cuda"),
-                                     u=torch.empty(B, self.F, dtype=torch.bfloat16, device="cuda"),
+                s["dec"].append(dict(x=x, pos=pos,
+                                     h=torch.empty(B, self.F, dtype=torch.bfloat16, device="cuda"),
                                      y=torch.empty(B, self.D, dtype=torch.bfloat16, device="cuda")))
             self.sets.append(s)
         self.rule = aal.row_rule(seq_len=self.seq_len)
@@ -145,9 +142,6 @@ class SwigluDecode:
         self.pin = dict(X=self.host_X.pin_memory(),
                         Y=torch.empty(self.M, self.D, dtype=torch.bfloat16).pin_memory(),
                         dec=[dict(x=d["x"].cpu().pin_memory(), pos=d["pos"].cpu().pin_memory(),
-                                  h=d["h"].cpu().pin_memory(),
-                                  g=torch.empty_like(d["g"], device="cpu").pin_memory(),
-                                  u=torch.empty_like(d["u"], device="cpu").pin_memory(),
                                   y=torch.empty_like(d["y"], device="cpu").pin_memory())
                              for d in self.sets[0]["dec"]])
 
@@ -164,20 +158,21 @@ class SwigluDecode:
         types = sorted(set(int(t) for t in pos % self.q))
         S = aal.aal_block_table(self.law, self.q)
         used = sum(1 for kk in range(self.q) for a in range(self.q) if any(S[t, kk, a] for t in types))
-        flops, byts = 0, 0
-        for din, dout in ((D, F), (D, F), (F, D)):
-            bi, bo = din // self.q, dout // self.q
-            n_blocks = sum(int(S[int(t) % self.q, kk, a]) for t in pos for kk in range(self.q) for a in range(self.q))
-            flops += 2 * bi * bo * n_blocks
-            byts += e * (used * bi * bo + B * (din + dout)) + 8 * B
-        return flops / 3, byts / 3  # mean over the three projections of a decode step
+        n_blocks = sum(int(S[int(t) % self.q, kk, a]) for t in pos for kk in range(self.q) for a in range(self.q))
+        if name.startswith("decode gate_up"):
+            bi, bo = D // self.q, F // self.q
+            # Wg and Wu blocks some entry uses, x in, h out, positions
+            return 2 * 2 * bi * bo * n_blocks, e * (2 * used * bi * bo + B * (D + F)) + 8 * B
+        bi, bo = F // self.q, D // self.q
+        return 2 * bi * bo * n_blocks, e * (used * bi * bo + B * (F + D)) + 8 * B
 
     def timing_slots(self):
         """(name, kernel kind) of every launch of a step, in launch order;
         launches that share a name are one kernel of the breakdown."""
         slots = [("gate_up", aal.AAL_KERNEL_GATE_UP), ("down", aal.AAL_KERNEL_PROJECT)]
         for B in self.decode_batches:
-            slots += [(f"decode B={B}", aal.AAL_KERNEL_DECODE)] * 3
+            slots += [(f"decode gate_up B={B}", aal.AAL_KERNEL_DECODE_GATE_UP),
+                      (f"decode down B={B}", aal.AAL_KERNEL_DECODE)]
         return slots
 
     def step(self, i, ev=None):
@@ -187,12 +182,11 @@ class SwigluDecode:
         mark(0)
         mark(1)
         aal.aal_swiglu_fwd(self.law, self.q, self.rule, s["X"], s["Wg"], s["Wu"], s["Wd"], s["H"], s["Y"])
-        j = 2
-        for d in s["dec"]:
-            for x, w, y in ((d["x"], s["Wg"], d["g"]), (d["x"], s["Wu"], d["u"]), (d["h"], s["Wd"], d["y"])):
-                mark(j)
-                aal.aal_decode_matvec(self.law, self.q, d["pos"], x, w, y)
-                j += 1
+        for j, d in enumerate(s["dec"]):
+            mark(2 + 2 * j)
+            mark(3 + 2 * j)
+            aal.aal_swiglu_decode(self.law, self.q, d["pos"], d["x"], s["Wg"], s["Wu"], s["Wd"],
+                                  d["h"], d["y"])
 
     def dense_step(self, i):
         s = self.sets[i % len(self.sets)]
@@ -200,8 +194,8 @@ class SwigluDecode:
         torch.matmul(s["X"], s["Wu"], out=s["H"])
         torch.matmul(s["H"], s["Wd"], out=s["Y"])
         for d in s["dec"]:
-            torch.matmul(d["x"], s["Wg"], out=d["g"])
-            torch.matmul(d["x"], s["Wu"], out=d["u"])
+            torch.matmul(d["x"], s["Wg"], out=d["h"])
+            torch.matmul(d["x"], s["Wu"], out=d["h"])
             torch.matmul(d["h"], s["Wd"], out=d["y"])
 
     def e2e_step(self, i):
@@ -211,18 +205,15 @@ class SwigluDecode:
         s["X"].copy_(p["X"], non_blocking=True)
         for d, hd in zip(s["dec"], p["dec"]):
             d["x"].copy_(hd["x"], non_blocking=True)
-            d["h"].copy_(hd["h"], non_blocking=True)
             d["pos"].copy_(hd["pos"], non_blocking=True)
         self.step(i)
         p["Y"].copy_(s["Y"], non_blocking=True)
         for d, hd in zip(s["dec"], p["dec"]):
-            hd["g"].copy_(d["g"], non_blocking=True)
-            hd["u"].copy_(d["u"], non_blocking=True)
             hd["y"].copy_(d["y"], non_blocking=True)
 
     def e2e_bytes(self):
-        h2d = self.M * self.D * 2 + sum(B * (self.D + self.F) * 2 + B * 8 for B in self.decode_batches)
-        d2h = self.M * self.D * 2 + sum(B * (2 * self.F + self.D) * 2 for B in self.decode_batches)
+        h2d = self.M * self.D * 2 + sum(B * self.D * 2 + B * 8 for B in self.decode_batches)
+        d2h = self.M * self.D * 2 + sum(B * self.D * 2 for B in self.decode_batches)
         return h2d, d2h
 
     # ---- oracle sample for the CPU baseline / reference arm
@@ -234,8 +225,7 @@ class SwigluDecode:
         st = inputs.Stream(100)
         dec = []
         for B in self.decode_batches:
-            dec.append((st.normal(B, self.D, 1.0, "bf16").f64, st.normal(B, self.F, 1.0, "bf16").f64,
-                        st.positions(B, self.seq_len)))
+            dec.append((st.normal(B, self.D, 1.0, "bf16").f64, st.positions(B, self.seq_len)))
         rows = min(rows, self.M)
         sel = np.arange(rows) * (self.M // rows)
         flops = (self.fwd_flops * rows) // self.M + self.dec_flops
@@ -243,13 +233,11 @@ class SwigluDecode:
         def run():
             oracle.swiglu_rows(self.law, self.q, types, s["X"].f64, s["Wg"].f64, s["Wu"].f64,
                                s["Wd"].f64, sel)
-            for x, h, pos in dec:
-                oracle.decode(self.law, self.q, pos, x, s["Wg"].f64)
-                oracle.decode(self.law, self.q, pos, x, s["Wu"].f64)
-                oracle.decode(self.law, self.q, pos, h, s["Wd"].f64)
+            for x, pos in dec:
+                oracle.swiglu_decode(self.law, self.q, pos, x, s["Wg"].f64, s["Wu"].f64, s["Wd"].f64)
 
         desc = (f"oracle SwiGLU forward on {rows} of {self.M} rows (evenly strided, all row types) "
-                f"+ the full decode matvecs B={'/'.join(map(str, self.decode_batches))}")
+                f"+ the full FFN decode steps B={'/'.join(map(str, self.decode_batches))}")
         return flops, run, desc
 
 

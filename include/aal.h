@@ -155,6 +155,27 @@ AAL_API aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* posi
                              aal_mat x, aal_mat W, aal_mat y, void* stream);
 
 /*
+ * Decode step of a whole algebraic SwiGLU FFN: the three decode rows of its
+ * projections with the activation between them (agihunt.info digest:
+ * decoding evaluates only the new position's row; SwiGLU figures, gate, up
+ * and down all algebraic with the same row types):
+ *   h = silu(x * Wg) (.) (x * Wu),   y = h * Wd,   silu(z) = z / (1 + e^-z)
+ * where each "*" is the row-typed product of entry b's row type
+ * positions[b] mod q.
+ *   positions: device int64 [B]; x [B, D]; Wg, Wu [D, F]; Wd [F, D];
+ *   h [B, F] (caller's workspace, overwritten with the activation, bf16 or
+ *   fp32 like the inputs); y [B, D] (overwritten).
+ * Two launches: gate, up and the activation in one kernel, then the down
+ * decode.  An entry with a negative position is skipped (its rows of h and
+ * y are not written) and the device status reports AAL_ERR_DEVICE_BOUNDS.
+ * Errors: AAL_ERR_INVALID_ARG for inconsistent shapes or a missing
+ * positions array, AAL_ERR_UNSUPPORTED for mixed dtypes.
+ */
+AAL_API aal_status aal_swiglu_decode(int32_t law, int32_t q, const int64_t* positions,
+                             aal_mat x, aal_mat Wg, aal_mat Wu, aal_mat Wd, aal_mat h,
+                             aal_mat y, void* stream);
+
+/*
  * Full (not row-typed) product of square block matrices, Z = X * W
  * (agihunt.info digest: fixed-block square product, and the quadratic
  * arithmetic when the block size stays fixed while q grows).
@@ -219,10 +240,13 @@ AAL_API int32_t aal_last_path(void);
  * Kinds: AAL_KERNEL_PROJECT (1, also the down projection inside
  * aal_swiglu_fwd), AAL_KERNEL_GATE_UP (2, the fused gate/up/SiLU kernel of
  * aal_swiglu_fwd), AAL_KERNEL_BWD_DX (3), AAL_KERNEL_BWD_DW (4),
- * AAL_KERNEL_SQUARE (5), AAL_KERNEL_DECODE (6).
+ * AAL_KERNEL_SQUARE (5), AAL_KERNEL_DECODE (6, also the down decode inside
+ * aal_swiglu_decode), AAL_KERNEL_DECODE_GATE_UP (7, the gate/up/SiLU decode
+ * kernel of aal_swiglu_decode).
  */
 enum { AAL_KERNEL_PROJECT = 1, AAL_KERNEL_GATE_UP = 2, AAL_KERNEL_BWD_DX = 3,
-       AAL_KERNEL_BWD_DW = 4, AAL_KERNEL_SQUARE = 5, AAL_KERNEL_DECODE = 6 };
+       AAL_KERNEL_BWD_DW = 4, AAL_KERNEL_SQUARE = 5, AAL_KERNEL_DECODE = 6,
+       AAL_KERNEL_DECODE_GATE_UP = 7 };
 AAL_API aal_status aal_set_timing_events(int32_t kernel, void* before, void* after);
 
 /* Number of kernels launched by compute calls on this thread since the last

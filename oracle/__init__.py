@@ -308,6 +308,17 @@ def decode(law: str, q: int, positions, x, W) -> np.ndarray:
     return project(law, q, row_types(law, q, positions), x, W)
 
 
+def swiglu_decode(law: str, q: int, positions, x, Wg, Wu, Wd):
+    """Decode step of the algebraic SwiGLU FFN: for each new token at absolute
+    position positions[b], its row of each projection with the activation in
+    between (agihunt.info digest: decoding evaluates the new position's row;
+    the FFN projections share the row types).  Returns (H, Y) in float64."""
+    G = decode(law, q, positions, x, Wg)
+    U = decode(law, q, positions, x, Wu)
+    H = silu(G) * U
+    return H, decode(law, q, positions, H, Wd)
+
+
 def mac_ratio(law: str, q: int) -> float:
     """Fraction of a dense projection's MACs that one row type performs."""
     return block_product_count(law, q, True) / float(q * q)

@@ -147,3 +147,28 @@ def run_decode(law, q, B, din, dout, dtype, seq_len=1536, seed=0, same_type=None
     path = aal.aal_last_path()
     ref = oracle.decode(law, q, pos, x.f64, W.f64)
     return oracle.rel_err(host64(y), ref), path
+
+
+def run_swiglu_decode(law, q, B, D, F, dtype, seq_len=1536, seed=0, same_type=None,
+                      policy=aal.AAL_PATH_AUTO):
+    s = inputs.Stream(seed)
+    x = s.normal(B, D, 1.0, dtype)
+    Wg = s.normal(D, F, D ** -0.5, dtype)
+    Wu = s.normal(D, F, D ** -0.5, dtype)
+    Wd = s.normal(F, D, F ** -0.5, dtype)
+    pos = s.positions(B, seq_len)
+    if same_type is not None:
+        pos = (pos - pos % q + same_type).astype(np.int64)
+    h = torch.full((B, F), float("nan"), dtype=x.t.dtype, device="cuda")
+    y = torch.full((B, D), float("nan"), dtype=x.t.dtype, device="cuda")
+    aal.aal_set_path_policy(policy)
+    try:
+        aal.aal_swiglu_decode(law, q, torch.from_numpy(pos).cuda(), x.t.cuda(), Wg.t.cuda(),
+                              Wu.t.cuda(), Wd.t.cuda(), h, y)
+        torch.cuda.synchronize()
+        path = aal.aal_last_path()
+    finally:
+        aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
+    assert aal.aal_get_device_status() == aal.AAL_OK
+    H, Y = oracle.swiglu_decode(law, q, pos, x.f64, Wg.f64, Wu.f64, Wd.f64)
+    return oracle.rel_err(host64(h), H), oracle.rel_err(host64(y), Y), path

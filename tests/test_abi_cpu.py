@@ -115,6 +115,14 @@ def test_other_calls_argument_errors(lib):
                                0, None) == aal.AAL_ERR_INVALID_ARG
     # decode: null positions with rows
     assert lib.aal_decode_matvec(0, 2, None, _m(FAKE, 4, 8), W, _m(FAKE, 4, 8), None) == aal.AAL_ERR_INVALID_ARG
+    # swiglu decode: Wd of the wrong shape, null positions, mixed dtypes
+    Wg = _m(FAKE, 8, 12)
+    assert lib.aal_swiglu_decode(0, 2, FAKE, _m(FAKE, 4, 8), Wg, Wg, _m(FAKE, 8, 12), _m(FAKE, 4, 12),
+                                 _m(FAKE, 4, 8), None) == aal.AAL_ERR_INVALID_ARG
+    assert lib.aal_swiglu_decode(0, 2, None, _m(FAKE, 4, 8), Wg, Wg, _m(FAKE, 12, 8), _m(FAKE, 4, 12),
+                                 _m(FAKE, 4, 8), None) == aal.AAL_ERR_INVALID_ARG
+    assert lib.aal_swiglu_decode(0, 2, FAKE, _m(FAKE, 4, 8), Wg, Wg, _m(FAKE, 12, 8), _m(FAKE, 4, 12),
+                                 _m(FAKE, 4, 8, dtype=aal.AAL_F32), None) == aal.AAL_ERR_UNSUPPORTED
     # square: not square / aliasing output
     assert lib.aal_square_product(0, 2, _m(FAKE, 8, 4), W, _m(FAKE + 4096, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
     assert lib.aal_square_product(0, 2, X := _m(FAKE, 8, 8), W, _m(FAKE, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
@@ -128,6 +136,8 @@ def test_empty_inputs_launch_nothing(lib):
     assert lib.aal_project_fwd(0, 2, rule, _m(None, 0, 8), _m(FAKE, 8, 8), _m(None, 0, 8), None) == aal.AAL_OK
     assert lib.aal_square_product(0, 2, _m(None, 0, 0), _m(None, 0, 0), _m(None, 0, 0), None) == aal.AAL_OK
     assert lib.aal_decode_matvec(0, 2, None, _m(None, 0, 8), _m(FAKE, 8, 8), _m(None, 0, 8), None) == aal.AAL_OK
+    assert lib.aal_swiglu_decode(0, 2, None, _m(None, 0, 8), _m(FAKE, 8, 12), _m(FAKE, 8, 12),
+                                 _m(FAKE, 12, 8), _m(None, 0, 12), _m(None, 0, 8), None) == aal.AAL_OK
     assert aal.aal_launch_count() == 0
 
 

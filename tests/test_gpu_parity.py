@@ -11,7 +11,8 @@ import oracle
 import associative_algebra_block_b200 as aal
 from associative_algebra_block_b200 import inputs
 
-from gpu_cases import TOL, host64, run_bwd, run_decode, run_project, run_square, run_swiglu
+from gpu_cases import (TOL, host64, run_bwd, run_decode, run_project, run_square, run_swiglu,
+                       run_swiglu_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -123,6 +124,51 @@ def test_decode_negative_position_tensor_core_kernel():
     keep = np.array([0, 2])
     ref = oracle.decode("Q", 2, pos[keep], x.f64[keep], W.f64)
     assert oracle.rel_err(got[keep], ref) <= TOL["bf16"]
+
+
+# Whole-FFN decode step (fused gate/up/SiLU, then the down decode): the c2
+# batches, a batch split into 128-entry launches, single row types, and the
+# general path (fp32; 32-column groups).
+@pytest.mark.parametrize("B", [1, 8, 64, 128, 200])
+def test_swiglu_decode_c2(B):
+    eh, ey, path = run_swiglu_decode("Q2xQ2", 4, B, 768, 1536, "bf16", seed=300 + B)
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+    assert path == aal.AAL_PATH_DECODE
+
+
+@pytest.mark.parametrize("t", [0, 3])
+def test_swiglu_decode_single_type(t):
+    eh, ey, _ = run_swiglu_decode("Q2xQ2", 4, 1, 768, 1536, "bf16", seed=310 + t, same_type=t)
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"], (eh, ey)
+
+
+@pytest.mark.parametrize("law,q,B,D,F,dtype,path", [
+    ("Q", 2, 5, 64, 128, "f32", aal.AAL_PATH_GENERAL),
+    ("Q", 4, 9, 128, 128, "bf16", aal.AAL_PATH_GENERAL),
+    ("Q", 16, 33, 2048, 1024, "bf16", aal.AAL_PATH_DECODE),
+])
+def test_swiglu_decode_other_shapes(law, q, B, D, F, dtype, path):
+    eh, ey, got = run_swiglu_decode(law, q, B, D, F, dtype, seed=320 + B)
+    assert eh <= TOL[dtype] and ey <= TOL[dtype], (eh, ey)
+    assert got == path
+
+
+def test_swiglu_decode_negative_position():
+    s = inputs.Stream(7)
+    x = s.normal(3, 128, 1.0, "bf16")
+    Wg, Wu = s.normal(128, 256, 0.1, "bf16"), s.normal(128, 256, 0.1, "bf16")
+    Wd = s.normal(256, 128, 0.06, "bf16")
+    pos = np.array([5, -2, 8], dtype=np.int64)
+    h = torch.full((3, 256), float("nan"), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((3, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    aal.aal_swiglu_decode("Q", 2, torch.from_numpy(pos).cuda(), x.t.cuda(), Wg.t.cuda(), Wu.t.cuda(),
+                          Wd.t.cuda(), h, y)
+    assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
+    gh, gy = host64(h), host64(y)
+    assert np.all(np.isnan(gh[1])) and np.all(np.isnan(gy[1]))
+    keep = np.array([0, 2])
+    H, Y = oracle.swiglu_decode("Q", 2, pos[keep], x.f64[keep], Wg.f64, Wu.f64, Wd.f64)
+    assert oracle.rel_err(gh[keep], H) <= TOL["bf16"] and oracle.rel_err(gy[keep], Y) <= TOL["bf16"]
 
 
 # -------------------------------------------------- Qwen3-8B-shaped Q_32

@@ -370,6 +370,35 @@ def test_swiglu_rows_match_full():
     assert np.array_equal(y2, Y[[3, 9]]) and np.array_equal(h2, H[[3, 9]])
 
 
+def test_swiglu_decode_is_the_prefill_row_at_that_position():
+    # a decode step at position p equals row p of the prefill SwiGLU of a
+    # sequence that contains it: the FFN is row-local and the row type comes
+    # from the position alone
+    s = inputs.Stream(97)
+    L = 12
+    X = s.normal(L, 8, 1.0, "f32").f64
+    Wg, Wu = s.normal(8, 16, 0.3, "f32").f64, s.normal(8, 16, 0.3, "f32").f64
+    Wd = s.normal(16, 8, 0.3, "f32").f64
+    H, Y = oracle.swiglu("Q2xQ2", 4, oracle.row_types("Q2xQ2", 4, np.arange(L)), X, Wg, Wu, Wd)
+    pos = np.array([7, 0, 11, 5, 5])
+    h, y = oracle.swiglu_decode("Q2xQ2", 4, pos, X[pos], Wg, Wu, Wd)
+    assert np.array_equal(h, H[pos]) and np.array_equal(y, Y[pos])
+
+
+def test_swiglu_decode_q1_is_dense_swiglu_and_gate_up_not_symmetric():
+    s = inputs.Stream(98)
+    x = s.normal(3, 8, 1.0, "f32").f64
+    Wg, Wu = s.normal(8, 12, 0.3, "f32").f64, s.normal(8, 12, 0.3, "f32").f64
+    Wd = s.normal(12, 8, 0.3, "f32").f64
+    h, y = oracle.swiglu_decode("Q", 1, np.array([4, 9, 2]), x, Wg, Wu, Wd)
+    G, U = x @ Wg, x @ Wu
+    hd = G / (1.0 + np.exp(-G)) * U
+    assert np.allclose(h, hd, rtol=1e-14) and np.allclose(y, hd @ Wd, rtol=1e-13)
+    # exchanging gate and up changes the result (silu is applied to the gate)
+    h2, _ = oracle.swiglu_decode("Q", 1, np.array([4, 9, 2]), x, Wu, Wg, Wd)
+    assert not np.allclose(h2, h)
+
+
 # --------------------------------------------------------------------------
 # Mutations planted in the oracle: each must trip at least one pin
 # --------------------------------------------------------------------------
