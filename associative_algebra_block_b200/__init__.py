@@ -35,12 +35,12 @@ AAL_TYPES_POSITION, AAL_TYPES_EXPLICIT = 0, 1
 AAL_PATH_AUTO, AAL_PATH_TENSOR, AAL_PATH_GENERAL, AAL_PATH_DECODE = 0, 1, 2, 3
 
 EXPORTS = ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd", "aal_decode_matvec",
-           "aal_swiglu_decode", "aal_square_product", "aal_block_table", "aal_block_product_count",
+           "aal_swiglu_decode", "aal_swiglu_bwd", "aal_square_product", "aal_block_table", "aal_block_product_count",
            "aal_get_device_status", "aal_status_string", "aal_set_path_policy",
            "aal_last_path", "aal_launch_count", "aal_version", "aal_set_timing_events")
 AAL_KERNEL_PROJECT, AAL_KERNEL_GATE_UP, AAL_KERNEL_BWD_DX = 1, 2, 3
 AAL_KERNEL_BWD_DW, AAL_KERNEL_SQUARE, AAL_KERNEL_DECODE = 4, 5, 6
-AAL_KERNEL_DECODE_GATE_UP = 7
+AAL_KERNEL_DECODE_GATE_UP, AAL_KERNEL_SWIGLU_BWD = 7, 8
 
 
 class AalError(RuntimeError):
@@ -80,6 +80,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
                                 AalMat, vp], i32),
             "aal_swiglu_decode": ([i32, i32, vp, AalMat, AalMat, AalMat, AalMat, AalMat, AalMat, vp],
                                   i32),
+            "aal_swiglu_bwd": ([i32, i32, AalRowTypeRule] + [AalMat] * 14 + [vp], i32),
             "aal_project_bwd": ([i32, i32, AalRowTypeRule, AalMat, AalMat, AalMat, AalMat, AalMat,
                                  i32, vp], i32),
             "aal_decode_matvec": ([i32, i32, vp, AalMat, AalMat, AalMat, vp], i32),
@@ -145,7 +146,9 @@ def row_rule(seq_len: int | None = None, pos_offset: int = 0,
     if types is not None:
         if types.dtype != torch.int32:
             raise ValueError("types must be int32")
-        return AalRowTypeRule(AAL_TYPES_EXPLICIT, 0, 0, types.data_ptr() if types.numel() else None)
+        rule = AalRowTypeRule(AAL_TYPES_EXPLICIT, 0, 0, types.data_ptr() if types.numel() else None)
+        rule._types = types  # the C struct holds only the pointer: keep the tensor alive with it
+        return rule
     if seq_len is None:
         raise ValueError("give seq_len or types")
     return AalRowTypeRule(AAL_TYPES_POSITION, int(seq_len), int(pos_offset), None)
@@ -186,6 +189,12 @@ def aal_decode_matvec(law, q, positions, x, W, y, stream=None):
         raise ValueError("positions must be int64")
     _check(load().aal_decode_matvec(_law(law), q, positions.data_ptr() if positions.numel() else None,
                                     mat(x), mat(W), mat(y), _stream(stream)), "aal_decode_matvec")
+
+
+def aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, G, U, dG, dU, dX, dWg, dWu, dWd, stream=None):
+    _check(load().aal_swiglu_bwd(_law(law), q, rule, *(mat(t) for t in (X, Wg, Wu, Wd, H, dY, G, U, dG,
+                                                                         dU, dX, dWg, dWu, dWd)),
+                                 _stream(stream)), "aal_swiglu_bwd")
 
 
 def aal_swiglu_decode(law, q, positions, x, Wg, Wu, Wd, h, y, stream=None):

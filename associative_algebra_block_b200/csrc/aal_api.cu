@@ -12,8 +12,8 @@ static thread_local long long t_launches = 0;
 void note_launch(int n) { t_launches += n; }
 void note_path(int path) { t_last_path = path; }
 
-static thread_local cudaEvent_t t_ev_before[8] = {};
-static thread_local cudaEvent_t t_ev_after[8] = {};
+static thread_local cudaEvent_t t_ev_before[16] = {};
+static thread_local cudaEvent_t t_ev_after[16] = {};
 
 // Records an event on ``s``; while ``s`` is being captured into a CUDA graph
 // the record becomes an event-record node, so the event still timestamps the
@@ -159,7 +159,7 @@ aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_m
   RowTypes rt = make_types(rule, q);
   int paths = 0;
   if (want_dx && M > 0 && din > 0) {
-    aal_status st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dY, W, dX, s); },
+    aal_status st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dY, W, dX, 0, s); },
                              [&] { return simt_project_bwd_dx(law, q, rt, dY, W, dX, s); });
     if (st != AAL_OK) return st;
     paths |= 1 << t_last_path;
@@ -172,6 +172,74 @@ aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_m
     paths |= 1 << t_last_path;
   }
   if (paths) note_path((paths & (1 << AAL_PATH_GENERAL)) ? AAL_PATH_GENERAL : AAL_PATH_TENSOR);
+  return AAL_OK;
+}
+
+aal_status aal_swiglu_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_mat X, aal_mat Wg,
+                          aal_mat Wu, aal_mat Wd, aal_mat H, aal_mat dY, aal_mat G, aal_mat U,
+                          aal_mat dG, aal_mat dU, aal_mat dX, aal_mat dWg, aal_mat dWu,
+                          aal_mat dWd, void* stream) {
+  const aal_mat* all[] = {&X, &Wg, &Wu, &Wd, &H, &dY, &G, &U, &dG, &dU, &dX, &dWg, &dWu, &dWd};
+  if (!valid_law(law, q)) return AAL_ERR_INVALID_ARG;
+  for (const aal_mat* m : all)
+    if (!valid_mat(*m)) return AAL_ERR_INVALID_ARG;
+  for (const aal_mat* m : all)
+    if (m->dtype != X.dtype) return AAL_ERR_UNSUPPORTED;
+  const long long M = X.rows, D = X.cols, F = Wg.cols;
+  auto is = [](const aal_mat& m, long long r, long long c) { return m.rows == r && m.cols == c; };
+  if (!is(Wg, D, F) || !is(Wu, D, F) || !is(Wd, F, D) || !is(H, M, F) || !is(dY, M, D) ||
+      !is(G, M, F) || !is(U, M, F) || !is(dG, M, F) || !is(dU, M, F) || !is(dX, M, D) ||
+      !is(dWg, D, F) || !is(dWu, D, F) || !is(dWd, F, D))
+    return AAL_ERR_INVALID_ARG;
+  if (D % q || F % q) return AAL_ERR_INVALID_ARG;
+  if (!valid_rule(rule, M)) return AAL_ERR_INVALID_ARG;
+  note_path(0);
+  if (D == 0 || F == 0) return AAL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  RowTypes rt = make_types(rule, q);
+  int paths = 0;
+  aal_status st;
+  auto note = [&] { paths |= 1 << t_last_path; };
+  if (M > 0) {
+    // 1. the gate and up pre-activations, recomputed
+    st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, X, Wg, G, s); },
+                  [&] { return simt_project(law, q, rt, X, Wg, G, s); });
+    if (st != AAL_OK) return st;
+    note();
+    st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, X, Wu, U, s); },
+                  [&] { return simt_project(law, q, rt, X, Wu, U, s); });
+    if (st != AAL_OK) return st;
+    note();
+    // 2. dH = dY through the down projection's transposed table, and the
+    //    SiLU' chain: dG = dH u silu'(g), dU = dH silu(g)
+    st = dispatch(AAL_KERNEL_SWIGLU_BWD, s,
+                  [&] { return tc_swiglu_bwd_dh(law, q, rt, M, dY, Wd, G, U, dG, dU, s); },
+                  [&] {
+                    aal_status e = simt_project_bwd_dx(law, q, rt, dY, Wd, dG, s);
+                    return e != AAL_OK ? e : simt_swiglu_bwd_act(q, rt, G, U, dG, dU, s);
+                  });
+    if (st != AAL_OK) return st;
+    note();
+    // 3. dX = dG Wg^T + dU Wu^T over the table
+    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dG, Wg, dX, 0, s); },
+                  [&] { return simt_project_bwd_dx(law, q, rt, dG, Wg, dX, s); });
+    if (st != AAL_OK) return st;
+    note();
+    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dU, Wu, dX, 1, s); },
+                  [&] { return simt_project_bwd_dx(law, q, rt, dU, Wu, dX, s, 1); });
+    if (st != AAL_OK) return st;
+    note();
+  }
+  // 4. weight gradients (zero when there are no rows)
+  const aal_mat* dw_in[3][3] = {{&X, &dG, &dWg}, {&X, &dU, &dWu}, {&H, &dY, &dWd}};
+  for (auto& t : dw_in) {
+    const aal_mat &A = *t[0], &B = *t[1], &O = *t[2];
+    st = dispatch(AAL_KERNEL_BWD_DW, s, [&] { return tc_project_bwd_dw(law, q, rt, M, A, B, O, 0, s); },
+                  [&] { return simt_project_bwd_dw(law, q, rt, A, B, O, 0, s); });
+    if (st != AAL_OK) return st;
+    note();
+  }
+  note_path((paths & (1 << AAL_PATH_GENERAL)) ? AAL_PATH_GENERAL : AAL_PATH_TENSOR);
   return AAL_OK;
 }
 
@@ -330,7 +398,7 @@ const char* aal_status_string(int32_t status) {
 }
 
 aal_status aal_set_timing_events(int32_t kernel, void* before, void* after) {
-  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_DECODE_GATE_UP) return AAL_ERR_INVALID_ARG;
+  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_SWIGLU_BWD) return AAL_ERR_INVALID_ARG;
   t_ev_before[kernel] = (cudaEvent_t)before;
   t_ev_after[kernel] = (cudaEvent_t)after;
   return AAL_OK;

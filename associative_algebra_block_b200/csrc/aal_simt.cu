@@ -76,7 +76,7 @@ __global__ void k_swiglu_gate_up(int law, int q, RowTypes rt, long long rows,
 template <typename T>
 __global__ void k_bwd_dx(int law, int q, RowTypes rt, long long rows, const T* __restrict__ dY,
                          long long ldy, const T* __restrict__ W, long long ldw, T* __restrict__ dX,
-                         long long ldx, int bi, int bo) {
+                         long long ldx, int bi, int bo, int accumulate) {
   const long long j = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long r = (long long)blockIdx.y * blockDim.y + threadIdx.y;
   const long long din = (long long)bi * q;
@@ -91,7 +91,27 @@ __global__ void k_bwd_dx(int law, int q, RowTypes rt, long long rows, const T* _
     const T* wr = W + j * ldw + (long long)k * bo;
     for (int c = 0; c < bo; ++c) acc = fmaf(ld_elem(dyr + c), ld_elem(wr + c), acc);
   }
+  if (accumulate) acc += ld_elem(dX + r * ldx + j);
   st_elem(dX + r * ldx + j, acc);
+}
+
+// SiLU' chain of the SwiGLU backward, elementwise on rows of a valid type:
+// dG holds dH on entry; dG = dH u silu'(g) and dU = dH silu(g) on exit, with
+// silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + e^-g).
+template <typename T>
+__global__ void k_swiglu_bwd_act(int q, RowTypes rt, long long rows, long long F,
+                                 const T* __restrict__ G, long long ldg, const T* __restrict__ U,
+                                 long long ldu, T* __restrict__ dG, long long lddg,
+                                 T* __restrict__ dU, long long lddu) {
+  const long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long r = (long long)blockIdx.y * blockDim.y + threadIdx.y;
+  if (c >= F || r >= rows) return;
+  if (row_type(rt, r) < 0) return;
+  const float g = ld_elem(G + r * ldg + c), u = ld_elem(U + r * ldu + c);
+  const float dh = ld_elem(dG + r * lddg + c);
+  const float sg = 1.f / (1.f + expf(-g));
+  st_elem(dU + r * lddu + c, dh * g * sg);
+  st_elem(dG + r * lddg + c, dh * u * sg * (1.f + g * (1.f - sg)));
 }
 
 // dW[j, c] (block (a, k)) = sum over rows r with a in S(t_r, k) of X[r, j] dY[r, c].
@@ -195,7 +215,7 @@ aal_status simt_swiglu_gate_up(int law, int q, const RowTypes& rt, const aal_mat
 }
 
 aal_status simt_project_bwd_dx(int law, int q, const RowTypes& rt, const aal_mat& dY,
-                               const aal_mat& W, const aal_mat& dX, cudaStream_t s) {
+                               const aal_mat& W, const aal_mat& dX, cudaStream_t s, int accumulate) {
   const long long rows = dY.rows, din = W.rows;
   const int bi = (int)(din / q), bo = (int)(W.cols / q);
   if (rows == 0 || din == 0) return AAL_OK;
@@ -204,11 +224,31 @@ aal_status simt_project_bwd_dx(int law, int q, const RowTypes& rt, const aal_mat
   dim3 grd = grid2(din, rows, blk);
   if (dY.dtype == AAL_F32)
     k_bwd_dx<float><<<grd, blk, 0, s>>>(law, q, rt, rows, (const float*)dY.ptr, dY.ld,
-                                        (const float*)W.ptr, W.ld, (float*)dX.ptr, dX.ld, bi, bo);
+                                        (const float*)W.ptr, W.ld, (float*)dX.ptr, dX.ld, bi, bo,
+                                        accumulate);
   else
     k_bwd_dx<__nv_bfloat16><<<grd, blk, 0, s>>>(law, q, rt, rows, (const __nv_bfloat16*)dY.ptr,
                                                 dY.ld, (const __nv_bfloat16*)W.ptr, W.ld,
-                                                (__nv_bfloat16*)dX.ptr, dX.ld, bi, bo);
+                                                (__nv_bfloat16*)dX.ptr, dX.ld, bi, bo, accumulate);
+  note_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+aal_status simt_swiglu_bwd_act(int q, const RowTypes& rt, const aal_mat& G, const aal_mat& U,
+                               const aal_mat& dG, const aal_mat& dU, cudaStream_t s) {
+  const long long rows = G.rows, F = G.cols;
+  if (rows == 0 || F == 0) return AAL_OK;
+  dim3 blk(32, 8);
+  if (!grid_ok(F, rows, blk)) return AAL_ERR_UNSUPPORTED;
+  dim3 grd = grid2(F, rows, blk);
+  if (G.dtype == AAL_F32)
+    k_swiglu_bwd_act<float><<<grd, blk, 0, s>>>(q, rt, rows, F, (const float*)G.ptr, G.ld,
+                                                (const float*)U.ptr, U.ld, (float*)dG.ptr, dG.ld,
+                                                (float*)dU.ptr, dU.ld);
+  else
+    k_swiglu_bwd_act<__nv_bfloat16><<<grd, blk, 0, s>>>(
+        q, rt, rows, F, (const __nv_bfloat16*)G.ptr, G.ld, (const __nv_bfloat16*)U.ptr, U.ld,
+        (__nv_bfloat16*)dG.ptr, dG.ld, (__nv_bfloat16*)dU.ptr, dU.ld);
   note_launch();
   return cuda_status(cudaGetLastError());
 }

@@ -109,6 +109,11 @@ struct Params {
   uint32_t tmem_cols;  // TMEM allocation (power of two)
   int swiglu;          // epilogue: silu(acc0) * acc1
   int accumulate;      // epilogue: out += acc (register path, no TMA store)
+  int swiglu_bwd;      // epilogue: acc is dH; with G, U at the same place write
+                       // dG = dH u silu'(g) to out and dU = dH silu(g) to out2
+  const __nv_bfloat16* g_in;
+  const __nv_bfloat16* u_in;
+  __nv_bfloat16* out2;
   int tma_store;       // epilogue: stage in shared memory and store with TMA
   __nv_bfloat16* out;
   long long ldo;
@@ -860,7 +865,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
           ++nstore;
         } else if (!p.swap) {
           const long long x = d.rbase + row_in_tile;
-          if (x < d.rlimit) {
+          if (x < d.rlimit && p.swiglu_bwd) {
+            // SiLU' chain of the SwiGLU backward on the dH tile in registers
+            const long long off = (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
+            const uint4 g0 = reinterpret_cast<const uint4*>(p.g_in + off)[0];
+            const uint4 g1 = reinterpret_cast<const uint4*>(p.g_in + off)[1];
+            const uint4 u0 = reinterpret_cast<const uint4*>(p.u_in + off)[0];
+            const uint4 u1 = reinterpret_cast<const uint4*>(p.u_in + off)[1];
+            const __nv_bfloat16* gb0 = reinterpret_cast<const __nv_bfloat16*>(&g0);
+            const __nv_bfloat16* gb1 = reinterpret_cast<const __nv_bfloat16*>(&g1);
+            const __nv_bfloat16* ub0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
+            const __nv_bfloat16* ub1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+            float du[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float g = __bfloat162float(j < 8 ? gb0[j] : gb1[j - 8]);
+              const float u = __bfloat162float(j < 8 ? ub0[j] : ub1[j - 8]);
+              const float sg = __fdividef(1.0f, 1.0f + __expf(-g));  // sigmoid(g)
+              du[j] = v[j] * g * sg;                                  // dH silu(g)
+              v[j] = v[j] * u * sg * (1.0f + g * (1.0f - sg));        // dH u silu'(g)
+            }
+            uint4 w[2];
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(w);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            reinterpret_cast<uint4*>(p.out + off)[0] = w[0];
+            reinterpret_cast<uint4*>(p.out + off)[1] = w[1];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) h[j] = __floats2bfloat162_rn(du[2 * j], du[2 * j + 1]);
+            reinterpret_cast<uint4*>(p.out2 + off)[0] = w[0];
+            reinterpret_cast<uint4*>(p.out2 + off)[1] = w[1];
+          } else if (x < d.rlimit) {
             __nv_bfloat16* dst = p.out + (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
             if (p.accumulate) {
               uint4 o0 = reinterpret_cast<const uint4*>(dst)[0];
@@ -1016,7 +1051,7 @@ static bool map_mn(CUtensorMap* m, const aal_mat& t, int qv, int aw, int extent,
 // Output map for the TMA-store epilogue: 32 rows x 16 columns per store
 // (32-byte swizzle), or 16 rows x 32 columns when TMEM lanes are columns.
 static bool out_map(Params& p, const aal_mat& out, int qv) {
-  p.tma_store = p.accumulate ? 0 : 1;
+  p.tma_store = (p.accumulate || p.swiglu_bwd) ? 0 : 1;
   if (!p.tma_store) return true;
   if (p.swap) return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 32, 16, 0);
   return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 16, 32, 32);
@@ -1318,10 +1353,17 @@ aal_status tc_swiglu_gate_up(int law, int q, const RowTypes& rt, long long rows,
   return tc_project_impl(law, q, rt, rows, X, Wg, &Wu, H, s);
 }
 
-aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
-                             const aal_mat& W, const aal_mat& dX, cudaStream_t s) {
+// dX of a row-typed projection; with ``act`` (G, U, dU) the SwiGLU
+// backward's SiLU' chain runs in the epilogue: dX is then dG (the gradient of
+// the gate pre-activation) and dU receives the gradient of the up projection.
+static aal_status bwd_dx_impl(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
+                              const aal_mat& W, const aal_mat& dX, int accumulate,
+                              const aal_mat* G, const aal_mat* U, const aal_mat* dU, cudaStream_t s) {
   if (!is_sm100() || !position_rule_ok(rt, q, rows)) return AAL_ERR_UNSUPPORTED;
   if (!tc_aligned(dY) || !tc_aligned(W) || !tc_aligned(dX)) return AAL_ERR_UNSUPPORTED;
+  if (G && (!tc_aligned(*G) || !tc_aligned(*U) || !tc_aligned(*dU) || G->ld != dX.ld ||
+            U->ld != dX.ld || dU->ld != dX.ld))
+    return AAL_ERR_UNSUPPORTED;
   const long long bi = W.rows / q, bo = W.cols / q;
   if (bi % 16 || bo % 16) return AAL_ERR_UNSUPPORTED;
   Params p;
@@ -1331,6 +1373,13 @@ aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows,
   p.bo = (int)bo;
   p.out = (__nv_bfloat16*)dX.ptr;
   p.ldo = dX.ld;
+  p.accumulate = accumulate ? 1 : 0;
+  if (G) {
+    p.swiglu_bwd = 1;
+    p.g_in = (const __nv_bfloat16*)G->ptr;
+    p.u_in = (const __nv_bfloat16*)U->ptr;
+    p.out2 = (__nv_bfloat16*)dU->ptr;
+  }
   const int n = pick_n(bi, 256);
   if (!n) return AAL_ERR_UNSUPPORTED;
   p.xr = 128;
@@ -1347,6 +1396,17 @@ aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows,
   p.n2 = q;
   p.n3 = (int)(bi / n);
   return launch<false, false, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+}
+
+aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
+                             const aal_mat& W, const aal_mat& dX, int accumulate, cudaStream_t s) {
+  return bwd_dx_impl(law, q, rt, rows, dY, W, dX, accumulate, nullptr, nullptr, nullptr, s);
+}
+
+aal_status tc_swiglu_bwd_dh(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
+                            const aal_mat& Wd, const aal_mat& G, const aal_mat& U,
+                            const aal_mat& dG, const aal_mat& dU, cudaStream_t s) {
+  return bwd_dx_impl(law, q, rt, rows, dY, Wd, dG, 0, &G, &U, &dU, s);
 }
 
 aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,

@@ -309,6 +309,92 @@ class ProjFwdBwd:
     e2e_step = None
 
 
+class SwigluFwdBwd:
+    """Algebraic SwiGLU FFN forward and backward (training step of one FFN):
+    aal_swiglu_fwd then aal_swiglu_bwd (G and U recomputed, the SiLU' chain
+    fused into the dH kernel, dX through both input projections, three weight
+    gradients)."""
+
+    def __init__(self, name, law, q, M, D, F, seq_len):
+        self.name, self.law, self.q, self.M, self.D, self.F, self.seq_len = name, law, q, M, D, F, seq_len
+        self.f_df = _exec_flops_proj(law, q, M, D, F)  # one D->F projection
+        self.f_fd = _exec_flops_proj(law, q, M, F, D)  # one F->D projection
+        # forward: gate, up, down; backward: dH, dX through Wg and Wu, dWg, dWu,
+        # dWd (the recomputation of G and U is extra work, not counted)
+        self.exec_flops = 3 * self.f_df + 3 * self.f_fd + 3 * self.f_df
+        self.dense_flops = 9 * 2 * M * D * F
+
+    def config(self):
+        return {"workload": f"{self.name}: {self.law} q={self.q} SwiGLU FFN D={self.D} F={self.F} "
+                            f"M={self.M}, forward + backward (dX, dWg, dWu, dWd); executed FLOPs "
+                            f"count the 9 row-typed products the chain rule needs, not the "
+                            f"recomputed G and U",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F}
+
+    def bytes_per_set(self):
+        e = 2
+        return e * (2 * 3 * self.D * self.F + self.M * (3 * self.D + 6 * self.F))
+
+    def setup(self, nsets, seed):
+        ins = inputs.swiglu_inputs(self.D, self.F, self.M, seed=seed, dtype="bf16", want_f64=False)
+        dY = inputs.Stream(seed + 7).normal(self.M, self.D, 1.0, "bf16", want_f64=False).t
+        M, D, F = self.M, self.D, self.F
+        self.sets = []
+        for _ in range(nsets):
+            t = {k: ins[k].t.cuda() for k in ("X", "Wg", "Wu", "Wd")}
+            t["dY"] = dY.cuda()
+            for k in ("H", "G", "U", "dG", "dU"):
+                t[k] = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+            t["Y"] = torch.empty(M, D, dtype=torch.bfloat16, device="cuda")
+            t["dX"] = torch.empty(M, D, dtype=torch.bfloat16, device="cuda")
+            for k in ("dWg", "dWu"):
+                t[k] = torch.empty(D, F, dtype=torch.bfloat16, device="cuda")
+            t["dWd"] = torch.empty(F, D, dtype=torch.bfloat16, device="cuda")
+            self.sets.append(t)
+        self.rule = aal.row_rule(seq_len=self.seq_len)
+
+    def kernel_model(self, name, sets):
+        M, D, F, e = self.M, self.D, self.F, 2
+        return {
+            "fwd gate_up": (2 * self.f_df, e * (M * D + 2 * D * F + M * F)),
+            "fwd down": (self.f_fd, e * (M * F + F * D + M * D)),
+            "bwd G recompute": (self.f_df, e * (M * D + D * F + M * F)),
+            "bwd dH + SiLU'": (self.f_fd, e * (M * D + F * D + 4 * M * F)),
+            "bwd dX (gate)": (self.f_df, e * (M * F + D * F + M * D)),
+            "bwd dWg": (self.f_df, e * (M * D + M * F + D * F)),
+        }[name]
+
+    def timing_slots(self):
+        return [("fwd gate_up", aal.AAL_KERNEL_GATE_UP), ("fwd down", aal.AAL_KERNEL_PROJECT),
+                ("bwd G recompute", aal.AAL_KERNEL_PROJECT), ("bwd dH + SiLU'", aal.AAL_KERNEL_SWIGLU_BWD),
+                ("bwd dX (gate)", aal.AAL_KERNEL_BWD_DX), ("bwd dWg", aal.AAL_KERNEL_BWD_DW)]
+
+    def step(self, i, ev=None):
+        t = self.sets[i % len(self.sets)]
+        mark = _marker(ev)
+        mark(0)
+        mark(1)
+        aal.aal_swiglu_fwd(self.law, self.q, self.rule, t["X"], t["Wg"], t["Wu"], t["Wd"], t["H"], t["Y"])
+        for j in range(2, 6):
+            mark(j)
+        aal.aal_swiglu_bwd(self.law, self.q, self.rule, t["X"], t["Wg"], t["Wu"], t["Wd"], t["H"], t["dY"],
+                           t["G"], t["U"], t["dG"], t["dU"], t["dX"], t["dWg"], t["dWu"], t["dWd"])
+
+    def dense_step(self, i):
+        t = self.sets[i % len(self.sets)]
+        torch.matmul(t["X"], t["Wg"], out=t["G"])
+        torch.matmul(t["X"], t["Wu"], out=t["U"])
+        torch.matmul(t["H"], t["Wd"], out=t["Y"])
+        torch.matmul(t["dY"], t["Wd"].t(), out=t["dG"])
+        torch.matmul(t["dG"], t["Wg"].t(), out=t["dX"])
+        torch.matmul(t["dU"], t["Wu"].t(), out=t["dX"])
+        torch.matmul(t["X"].t(), t["dG"], out=t["dWg"])
+        torch.matmul(t["X"].t(), t["dU"], out=t["dWu"])
+        torch.matmul(t["H"].t(), t["dY"], out=t["dWd"])
+
+    e2e_step = None
+
+
 class Square:
     def __init__(self, name, law, q, n):
         self.name, self.law, self.q, self.n = name, law, q, n
@@ -354,6 +440,7 @@ WORKLOADS = {
                                w_sigma_rule="D", decode_batches=()),
     "c4": lambda: ProjFwdBwd("Qwen3-30B-A3B-expert-shaped FFN", "Q", 16, 2048, 2048, 768, 2048),
     "c5": lambda: Square("fixed-block square", "Q", 256, 32768),
+    "c4-swiglu": lambda: SwigluFwdBwd("Qwen3-30B-A3B-expert-shaped SwiGLU FFN", "Q", 16, 2048, 2048, 768, 2048),
 }
 
 

@@ -144,6 +144,30 @@ AAL_API aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rul
                            void* stream);
 
 /*
+ * Backward of aal_swiglu_fwd (agihunt.info digest, SwiGLU figures and the
+ * kernel table's backward row; the composition of the projection backward
+ * with the derivative of silu(g) u):
+ *   G = X*Wg, U = X*Wu (recomputed), dH = dY through Wd's transposed table,
+ *   dG = dH (.) U (.) silu'(G), dU = dH (.) silu(G),
+ *   dX = dG through Wg's transposed table + dU through Wu's,
+ *   dWg = X^T-typed dG, dWu = X^T-typed dU, dWd = H^T-typed dY,
+ * with silu'(g) = s (1 + g (1 - s)), s = 1 / (1 + e^-g), every product
+ * row-typed with the same rule as the forward.
+ *   X [M, D], Wg, Wu [D, F], Wd [F, D], H [M, F] (the forward's activation),
+ *   dY [M, D]: inputs.  G, U, dG, dU [M, F]: caller's workspace, overwritten
+ *   (on return they hold the pre-activations and their gradients).
+ *   dX [M, D], dWg, dWu [D, F], dWd [F, D]: overwritten.
+ * The SiLU' chain runs in the epilogue of the dH kernel on the tensor-core
+ * path; the general path uses a separate elementwise kernel.  Errors:
+ * AAL_ERR_INVALID_ARG for inconsistent shapes, AAL_ERR_UNSUPPORTED for mixed
+ * dtypes.
+ */
+AAL_API aal_status aal_swiglu_bwd(int32_t law, int32_t q, aal_row_type_rule rule,
+                          aal_mat X, aal_mat Wg, aal_mat Wu, aal_mat Wd, aal_mat H,
+                          aal_mat dY, aal_mat G, aal_mat U, aal_mat dG, aal_mat dU,
+                          aal_mat dX, aal_mat dWg, aal_mat dWu, aal_mat dWd, void* stream);
+
+/*
  * Decode step: one new token per batch entry (agihunt.info digest: decoding
  * evaluates only the new position's row, as a matrix-vector product with its
  * own kernel).
@@ -242,11 +266,13 @@ AAL_API int32_t aal_last_path(void);
  * aal_swiglu_fwd), AAL_KERNEL_BWD_DX (3), AAL_KERNEL_BWD_DW (4),
  * AAL_KERNEL_SQUARE (5), AAL_KERNEL_DECODE (6, also the down decode inside
  * aal_swiglu_decode), AAL_KERNEL_DECODE_GATE_UP (7, the gate/up/SiLU decode
- * kernel of aal_swiglu_decode).
+ * kernel of aal_swiglu_decode), AAL_KERNEL_SWIGLU_BWD (8, the dH kernel of
+ * aal_swiglu_bwd with the SiLU' chain; aal_swiglu_bwd's other launches use
+ * the PROJECT, BWD_DX and BWD_DW kinds).
  */
 enum { AAL_KERNEL_PROJECT = 1, AAL_KERNEL_GATE_UP = 2, AAL_KERNEL_BWD_DX = 3,
        AAL_KERNEL_BWD_DW = 4, AAL_KERNEL_SQUARE = 5, AAL_KERNEL_DECODE = 6,
-       AAL_KERNEL_DECODE_GATE_UP = 7 };
+       AAL_KERNEL_DECODE_GATE_UP = 7, AAL_KERNEL_SWIGLU_BWD = 8 };
 AAL_API aal_status aal_set_timing_events(int32_t kernel, void* before, void* after);
 
 /* Number of kernels launched by compute calls on this thread since the last

@@ -296,6 +296,25 @@ def swiglu(law: str, q: int, types, X, Wg, Wu, Wd):
     return H, project(law, q, types, H, Wd)
 
 
+def swiglu_bwd(law: str, q: int, types, X, Wg, Wu, Wd, dY):
+    """Gradients of L = <dY, Y> for the algebraic SwiGLU FFN (Y from
+    ``swiglu``): chain rule through the down projection, the product
+    silu(G) . U (silu'(g) = s (1 + g (1 - s)), s the logistic function) and
+    the two input projections, each through ``project_bwd``.
+    Returns (dX, dWg, dWu, dWd) in float64."""
+    X = np.asarray(X, dtype=np.float64)
+    G = project(law, q, types, X, Wg)
+    U = project(law, q, types, X, Wu)
+    H = silu(G) * U
+    dH, dWd = project_bwd(law, q, types, H, Wd, dY)
+    sg = 1.0 / (1.0 + np.exp(-G))
+    dG = dH * U * sg * (1.0 + G * (1.0 - sg))
+    dU = dH * silu(G)
+    dXg, dWg = project_bwd(law, q, types, X, Wg, dG)
+    dXu, dWu = project_bwd(law, q, types, X, Wu, dU)
+    return dXg + dXu, dWg, dWu, dWd
+
+
 def swiglu_rows(law: str, q: int, types, X, Wg, Wu, Wd, rows):
     """SwiGLU on a subset of rows (the FFN is row-local)."""
     rows = np.asarray(rows, dtype=np.int64)

@@ -172,3 +172,36 @@ def run_swiglu_decode(law, q, B, D, F, dtype, seq_len=1536, seed=0, same_type=No
     assert aal.aal_get_device_status() == aal.AAL_OK
     H, Y = oracle.swiglu_decode(law, q, pos, x.f64, Wg.f64, Wu.f64, Wd.f64)
     return oracle.rel_err(host64(h), H), oracle.rel_err(host64(y), Y), path
+
+
+def run_swiglu_bwd(law, q, M, D, F, dtype, seq_len=None, seed=0, explicit=False,
+                   policy=aal.AAL_PATH_AUTO):
+    ins = inputs.swiglu_inputs(D, F, M, seed=seed, dtype=dtype)
+    X, Wg, Wu, Wd = (dev(ins[k]) for k in ("X", "Wg", "Wu", "Wd"))
+    dYd = inputs.Stream(seed + 7).normal(M, D, 1.0, dtype)
+    dY = dev(dYd)
+    if explicit:
+        tv = inputs.Stream(seed + 1).labels(M, q)
+        types_t = torch.from_numpy(tv).cuda()  # the rule holds only its pointer
+        rule = aal.row_rule(types=types_t)
+        types = tv.astype(np.int64)
+    else:
+        seq_len = seq_len or M
+        rule = aal.row_rule(seq_len=seq_len)
+        types = packed_types(law, q, M, seq_len)
+    H = torch.empty(M, F, dtype=X.dtype, device="cuda")
+    Y = torch.empty(M, D, dtype=X.dtype, device="cuda")
+    aal.aal_set_path_policy(policy)
+    try:
+        aal.aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y)
+        ws = [torch.full((M, F), float("nan"), dtype=X.dtype, device="cuda") for _ in range(4)]
+        outs = [torch.full(t.shape, float("nan"), dtype=X.dtype, device="cuda") for t in (X, Wg, Wu, Wd)]
+        aal.aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, *ws, *outs)
+        torch.cuda.synchronize()
+        path = aal.aal_last_path()
+    finally:
+        aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
+    assert aal.aal_get_device_status() == aal.AAL_OK
+    ref = oracle.swiglu_bwd(law, q, types, ins["X"].f64, ins["Wg"].f64, ins["Wu"].f64, ins["Wd"].f64,
+                            dYd.f64)
+    return [oracle.rel_err(host64(o), r) for o, r in zip(outs, ref)], path

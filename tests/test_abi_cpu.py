@@ -123,6 +123,11 @@ def test_other_calls_argument_errors(lib):
                                  _m(FAKE, 4, 8), None) == aal.AAL_ERR_INVALID_ARG
     assert lib.aal_swiglu_decode(0, 2, FAKE, _m(FAKE, 4, 8), Wg, Wg, _m(FAKE, 12, 8), _m(FAKE, 4, 12),
                                  _m(FAKE, 4, 8, dtype=aal.AAL_F32), None) == aal.AAL_ERR_UNSUPPORTED
+    # swiglu bwd: dWd of the wrong shape, mixed dtypes
+    m_mf, m_md = _m(FAKE, 16, 12), _m(FAKE, 16, 8)
+    good = [X, Wg, Wg, _m(FAKE, 12, 8), m_mf, m_md, m_mf, m_mf, m_mf, m_mf, m_md, Wg, Wg]
+    assert lib.aal_swiglu_bwd(0, 2, rule, *good, _m(FAKE, 8, 12), None) == aal.AAL_ERR_INVALID_ARG
+    assert lib.aal_swiglu_bwd(0, 2, rule, *good, _m(FAKE, 12, 8, dtype=aal.AAL_F32), None) == aal.AAL_ERR_UNSUPPORTED
     # square: not square / aliasing output
     assert lib.aal_square_product(0, 2, _m(FAKE, 8, 4), W, _m(FAKE + 4096, 8, 8), None) == aal.AAL_ERR_INVALID_ARG
     assert lib.aal_square_product(0, 2, X := _m(FAKE, 8, 8), W, _m(FAKE, 8, 8), None) == aal.AAL_ERR_INVALID_ARG

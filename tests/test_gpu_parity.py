@@ -11,8 +11,8 @@ import oracle
 import associative_algebra_block_b200 as aal
 from associative_algebra_block_b200 import inputs
 
-from gpu_cases import (TOL, host64, run_bwd, run_decode, run_project, run_square, run_swiglu,
-                       run_swiglu_decode)
+from gpu_cases import (TOL, dev, host64, run_bwd, run_decode, run_project, run_square, run_swiglu,
+                       run_swiglu_bwd, run_swiglu_decode)
 
 pytestmark = pytest.mark.gpu
 
@@ -169,6 +169,36 @@ def test_swiglu_decode_negative_position():
     keep = np.array([0, 2])
     H, Y = oracle.swiglu_decode("Q", 2, pos[keep], x.f64[keep], Wg.f64, Wu.f64, Wd.f64)
     assert oracle.rel_err(gh[keep], H) <= TOL["bf16"] and oracle.rel_err(gy[keep], Y) <= TOL["bf16"]
+
+
+# SwiGLU backward (dX, dWg, dWu, dWd): the expert-shaped FFN on the
+# tensor-core path with the SiLU' chain in the dH epilogue, the pilot law,
+# and the general path (fp32; explicit row types).
+@pytest.mark.parametrize("law,q,M,D,F,dtype,explicit,path", [
+    ("Q", 16, 2048, 2048, 768, "bf16", False, aal.AAL_PATH_TENSOR),
+    ("Q2xQ2", 4, 1024, 768, 1536, "bf16", False, aal.AAL_PATH_TENSOR),
+    ("Q", 2, 64, 64, 128, "f32", False, aal.AAL_PATH_GENERAL),
+    ("Q", 4, 96, 128, 256, "bf16", True, aal.AAL_PATH_GENERAL),
+])
+def test_swiglu_bwd(law, q, M, D, F, dtype, explicit, path):
+    errs, got = run_swiglu_bwd(law, q, M, D, F, dtype, seed=M + q, explicit=explicit)
+    assert max(errs) <= TOL[dtype], errs
+    assert got == path
+
+
+def test_swiglu_autograd_wrapper():
+    from associative_algebra_block_b200.autograd import swiglu
+    ins = inputs.swiglu_inputs(256, 512, 512, seed=3, dtype="bf16")
+    t = [dev(ins[k]).requires_grad_(True) for k in ("X", "Wg", "Wu", "Wd")]
+    dYd = inputs.Stream(9).normal(512, 256, 1.0, "bf16")
+    Y = swiglu("Q2xQ2", 4, aal.row_rule(seq_len=512), *t)
+    Y.backward(dev(dYd))
+    types = oracle.row_types("Q2xQ2", 4, np.arange(512))
+    _, Yref = oracle.swiglu("Q2xQ2", 4, types, *(ins[k].f64 for k in ("X", "Wg", "Wu", "Wd")))
+    assert oracle.rel_err(host64(Y.detach()), Yref) <= TOL["bf16"]
+    ref = oracle.swiglu_bwd("Q2xQ2", 4, types, *(ins[k].f64 for k in ("X", "Wg", "Wu", "Wd")), dYd.f64)
+    for ti, r in zip(t, ref):
+        assert oracle.rel_err(host64(ti.grad), r) <= TOL["bf16"]
 
 
 # -------------------------------------------------- Qwen3-8B-shaped Q_32

@@ -370,6 +370,49 @@ def test_swiglu_rows_match_full():
     assert np.array_equal(y2, Y[[3, 9]]) and np.array_equal(h2, H[[3, 9]])
 
 
+def test_swiglu_bwd_q1_matches_torch_autograd():
+    # at q = 1 the algebraic FFN is the dense one; torch's float64 autograd on
+    # the CPU differentiates it independently of the oracle's chain rule
+    import torch
+    s = inputs.Stream(99)
+    X = s.normal(5, 8, 1.0, "f32").f64
+    Wg, Wu = s.normal(8, 12, 0.4, "f32").f64, s.normal(8, 12, 0.4, "f32").f64
+    Wd = s.normal(12, 8, 0.4, "f32").f64
+    dY = s.normal(5, 8, 1.0, "f32").f64
+    got = oracle.swiglu_bwd("Q", 1, np.zeros(5, np.int64), X, Wg, Wu, Wd, dY)
+    t = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (X, Wg, Wu, Wd)]
+    Y = (torch.nn.functional.silu(t[0] @ t[1]) * (t[0] @ t[2])) @ t[3]
+    (Y * torch.tensor(dY)).sum().backward()
+    for g, ti in zip(got, t):
+        assert np.allclose(g, ti.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("law,q", [("Q2xQ2", 4), ("Q", 3)])
+def test_swiglu_bwd_finite_differences(law, q):
+    s = inputs.Stream(100 + q)
+    M, D, F = 2 * q, 2 * q, 3 * q
+    X = s.normal(M, D, 1.0, "f32").f64
+    Wg, Wu = s.normal(D, F, 0.5, "f32").f64, s.normal(D, F, 0.5, "f32").f64
+    Wd = s.normal(F, D, 0.5, "f32").f64
+    dY = s.normal(M, D, 1.0, "f32").f64
+    types = np.arange(M) % q
+    grads = oracle.swiglu_bwd(law, q, types, X, Wg, Wu, Wd, dY)
+    args = [X, Wg, Wu, Wd]
+
+    def loss(a):
+        return float(np.sum(dY * oracle.swiglu(law, q, types, *a)[1]))
+
+    h = 1e-6
+    for which in range(4):
+        for (r, c) in ((0, 0), (1, 2), (M - 1 if which == 0 else 2, 1)):
+            up = [a.copy() for a in args]
+            dn = [a.copy() for a in args]
+            up[which][r, c] += h
+            dn[which][r, c] -= h
+            fd = (loss(up) - loss(dn)) / (2 * h)
+            assert abs(fd - grads[which][r, c]) < 1e-6 * max(1.0, abs(fd))
+
+
 def test_swiglu_decode_is_the_prefill_row_at_that_position():
     # a decode step at position p equals row p of the prefill SwiGLU of a
     # sequence that contains it: the FFN is row-local and the row type comes
