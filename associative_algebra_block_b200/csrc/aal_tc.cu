@@ -865,7 +865,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
           ++nstore;
         } else if (!p.swap) {
           const long long x = d.rbase + row_in_tile;
-          if (x < d.rlimit && p.swiglu_bwd) {
+          // the SiLU' chain exists only in the dX instantiation (K-major A and B, one B)
+          constexpr bool kDxKernel = !A_MN && !B_MN && DUAL == 0 && !PAIR;
+          if (kDxKernel && x < d.rlimit && p.swiglu_bwd) {
             // SiLU' chain of the SwiGLU backward on the dH tile in registers
             const long long off = (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
             const uint4 g0 = reinterpret_cast<const uint4*>(p.g_in + off)[0];
