@@ -43,10 +43,14 @@ L2_BYTES = 126 * 2 ** 20
 # kernel the bench reports null.
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
-    ("c2", "gate_up"): ("7b4dbbdd970c1f53d959e716da9b8e65cce5c962aa7fc6f0820cdda6ddad05b2",
-                        23669504 + 1120256, "aal_tc.cu"),
-    ("c2", "down"): ("7b4dbbdd970c1f53d959e716da9b8e65cce5c962aa7fc6f0820cdda6ddad05b2",
-                     40178176 + 857856, "aal_tc.cu"),
+    ("c2", "gate_up"): ("c7c9977d016b0d3276cbea16de8334b8b64d0d7d539a4823ff811096d07ad88a",
+                        23666944 + 1915136, "aal_tc.cu"),
+    ("c2", "down"): ("c7c9977d016b0d3276cbea16de8334b8b64d0d7d539a4823ff811096d07ad88a",
+                     40179200 + 2312960, "aal_tc.cu"),
+    ("c2", "decode gate_up B=64"): ("0b5046ce4d0b0f216ae803d6612f53ea6f83636fb5dd818067011eed53c4bfe4",
+                                    4851968, "aal_decode.cu"),
+    ("c2", "decode down B=64"): ("0b5046ce4d0b0f216ae803d6612f53ea6f83636fb5dd818067011eed53c4bfe4",
+                                 2586112, "aal_decode.cu"),
 }
 
 
