@@ -3,14 +3,19 @@
 // position's row, as a matrix-vector product with a kernel of its own).
 //
 // The work is a stream over the weight rows that some entry of the batch
-// needs: a weight row is loaded only when some entry of a CTA's batch tile
-// needs its group for the thread's columns, so one row type touches
-// (2q-1)/q^2 of W (9/16 for Q2xQ2) in arithmetic.  k_decode_split (weight
-// rows split across a thread-block cluster, activations staged in shared
-// memory) serves aligned bf16 weights whose output groups are multiples of
-// 64 columns; k_decode_vec (16-byte vector loads, rows loaded only when some
-// entry needs them) the other aligned ones, fp32 included; k_decode is the
-// scalar fallback.
+// needs: a weight block is loaded only when some entry's table row uses it,
+// so one row type touches (2q-1)/q^2 of W (9/16 for Q2xQ2).  Kernels, in the
+// order the dispatcher tries them:
+//   k_decode_mma (bf16, <= 256 entries, 64-column output groups): warp-level
+//     tensor-core MMAs, split-K over an 8-CTA cluster (clusters of 2, 4 and
+//     16 measured slower on B200), also the fused gate/up/SiLU step of a
+//     SwiGLU FFN;
+//   k_decode_typed (bf16, 32-column groups): a CTA per column slab and row
+//     type streams only the rows of S(t, k);
+//   k_decode_split (bf16, 64-column groups): weight rows split across a
+//     cluster, activations staged in shared memory;
+//   k_decode_vec (16-byte vector loads, fp32 included) and k_decode (scalar)
+//     for everything else.
 #include <cooperative_groups.h>
 #include <limits.h>
 #include <stdlib.h>
@@ -650,9 +655,9 @@ static cudaError_t launch_typed(int law, int q, const int64_t* positions, int B,
 // entry of the batch needs are neither loaded nor multiplied, so HBM traffic
 // stays the table's.  CTA (column tile, z) owns 64 output columns (inside one
 // output group k) and the K slice z of the weight rows; the slices of one
-// column tile form a thread-block cluster and their fp32 partial products
-// meet in distributed shared memory, each CTA summing and writing a share of
-// the batch rows.
+// column tile form a thread-block cluster and each pushes its fp32 partial
+// products into the shared memory of the CTA that owns the entry, which sums
+// and writes it.
 // Operand orientation: the MMA's M is the 64 output columns (A = W^T, read
 // from the row-major weight tile with ldmatrix .trans), N the batch entries
 // (B = X^T, rows of X), K the weight rows.

@@ -777,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     const int quarter = warp & 3;             // TMEM lanes this warp may read
     const int half = (warp - 2) / 4;          // which of the 16-column chunks it drains
     const int row_in_tile = quarter * 32 + lane;
-    // two 1 KB staging buffers per epilogue warp, after the pipeline stages
+    // two 1 KB TMA-store staging buffers per epilogue warp, after the pipeline stages
     const uint32_t stage_buf = smem0 + S * p.stage_bytes + (warp - 2) * 2048;
     uint32_t nstore = 0;
     uint32_t tl = 0;
