@@ -92,3 +92,23 @@ def test_reference_arm_rank0_prints_one_contract_line():
         assert k in d
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_bench_kernel_models_add_up_to_the_step():
+    # the per-launch FLOP models of the c2 step's kernels sum to the step's
+    # executed FLOPs (so a kernel's roofline and the step's value agree)
+    import torch
+    import bench
+    from associative_algebra_block_b200 import inputs
+    wl = bench.WORKLOADS["c2"]()
+    st = inputs.Stream(100)
+    dec = [{"pos": torch.from_numpy(st.positions(B, wl.seq_len))} for B in wl.decode_batches]
+    total = 0
+    for name, _ in wl.timing_slots():
+        flops, byts = wl.kernel_model(name, [{"dec": dec}])
+        assert byts > 0
+        total += flops
+    assert total == wl.exec_flops
+    # c4-swiglu: the six timed launches are a subset of the step's work
+    w4 = bench.WORKLOADS["c4-swiglu"]()
+    assert sum(w4.kernel_model(n, None)[0] for n, _ in w4.timing_slots()) < w4.exec_flops
