@@ -161,3 +161,22 @@ def test_path_policy_round_trip(lib):
     with pytest.raises(aal.AalError):
         aal.aal_set_path_policy(7)
     assert aal.aal_version() >= 100
+
+
+def test_plain_c_program_uses_the_boundary(lib, tmp_path):
+    # the header and library work from C with no Python or torch in between
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    exe = tmp_path / "abi_host"
+    pkg = os.path.dirname(aal.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c11", "-O1", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c", "abi_host.c"), "-o", str(exe),
+                        "-L", pkg, "-l:libaal.so", "-Wl,-rpath," + pkg],
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "table ok" in r.stdout and "counts ok" in r.stdout and "argument check ok" in r.stdout
