@@ -664,13 +664,15 @@ static cudaError_t launch_typed(int law, int q, const int64_t* positions, int B,
 constexpr int kMmaCols = 64;      // output columns per CTA
 constexpr int kMmaMaxB = 256;     // batch entries per launch
 constexpr int kMmaMaxBGU = 128;   // batch entries per launch of the fused gate/up kernel
-constexpr int kMmaKc = 192;       // weight rows staged per round
+constexpr int kMmaKc = 192;       // weight rows staged per round, at most
 constexpr int kMmaWStride = 72;   // staged weight row: 64 columns + 8 pad (144 bytes)
 constexpr int kMmaPStride = 68;   // fp32 partial row: 64 columns + 4 pad
 
-// Shared memory of the staging area (weight rows + activations), 16-byte multiple.
-__host__ __device__ inline size_t mma_stage_bytes(int Bp, int nw) {
-  return (size_t)nw * kMmaKc * kMmaWStride * 2 + (size_t)Bp * (kMmaKc + 8) * 2;
+// Shared memory of the staging area (weight rows + activations) for rounds of
+// kcr weight rows (a multiple of 16), 16-byte multiple.  Sizing it by the
+// slice rather than the largest round lets two or three CTAs share an SM.
+__host__ __device__ inline size_t mma_stage_bytes(int Bp, int nw, int kcr) {
+  return (size_t)nw * kcr * kMmaWStride * 2 + (size_t)Bp * (kcr + 8) * 2;
 }
 __device__ __forceinline__ uint32_t dec_smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -735,12 +737,13 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   const int ntiles = Bp >> 3;
   const int cl = (int)gridDim.z;
   const int rows_own = (Bp + cl - 1) / cl;  // entries owned per CTA (upper bound)
-  const int xs_stride = kMmaKc + 8;         // staged activation row, bf16
+  const int kcr = min(kMmaKc, slice);      // weight rows per staging round
+  const int xs_stride = kcr + 8;            // staged activation row, bf16
   constexpr int NW = GU ? 2 : 1;  // weight tiles staged per round
   __nv_bfloat16* Ws = reinterpret_cast<__nv_bfloat16*>(dsm);
-  __nv_bfloat16* Xs = Ws + NW * kMmaKc * kMmaWStride;
+  __nv_bfloat16* Xs = Ws + NW * kcr * kMmaWStride;
   // receive area: [operand][source rank][owned entry][64 columns] fp32, after staging
-  float* R = reinterpret_cast<float*>(dsm + mma_stage_bytes(Bp, NW));
+  float* R = reinterpret_cast<float*>(dsm + mma_stage_bytes(Bp, NW, kcr));
   const int g0 = ks0 / bi, ng = (ks0 + slice - 1) / bi - g0 + 1;
 
   // the position of entry tid is in flight while the copies are issued
@@ -754,7 +757,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
         cp_async16(dec_smem_u32(Ws + r * kMmaWStride + ch * 8),
                    W + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
         if (GU)
-          cp_async16(dec_smem_u32(Ws + (kMmaKc + r) * kMmaWStride + ch * 8),
+          cp_async16(dec_smem_u32(Ws + (kcr + r) * kMmaWStride + ch * 8),
                      W2 + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
       }
     }
@@ -771,7 +774,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   };
 
   // round 0's copies go out first
-  stage(ks0, min(kMmaKc, slice), true);
+  stage(ks0, kcr, true);
 
   // 1. row type of every entry (-1 for padding and invalid positions) and
   //    the set of types present
@@ -817,8 +820,8 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
     my_t[j] = n < Bp ? s_type[n] : -1;
   }
 
-  for (int kc = 0; kc < slice; kc += kMmaKc) {
-    const int rows = min(kMmaKc, slice - kc);
+  for (int kc = 0; kc < slice; kc += kcr) {
+    const int rows = min(kcr, slice - kc);
     const int r0 = ks0 + kc;  // first weight row of this round
     if (kc > 0) stage(r0, rows, false);
     asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -848,7 +851,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
       const int acol = mt * 16 + (((lane >> 3) & 1) << 3);
 #pragma unroll
       for (int o = 0; o < NW; ++o)
-        ldsm_x4_trans(dec_smem_u32(Ws + (o * kMmaKc + arow) * kMmaWStride + acol), af[o]);
+        ldsm_x4_trans(dec_smem_u32(Ws + (o * kcr + arow) * kMmaWStride + acol), af[o]);
       uint32_t bf[NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -867,7 +870,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
           for (int o = 0; o < NW; ++o) mma_bf16_16816(acc[o][j], af[o], bf[j]);
         }
     }
-    if (kc + kMmaKc < slice) __syncthreads();  // staging is refilled next round
+    if (kc + kcr < slice) __syncthreads();  // staging is refilled next round
   }
   // 4. push the fp32 partials to their owners: entry n -> CTA n mod cl,
   //    slot [this rank][n / cl]
@@ -924,9 +927,9 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   }
 }
 
-static size_t mma_smem_bytes(int Bp, int cl, int nw) {
+static size_t mma_smem_bytes(int Bp, int cl, int nw, int kcr) {
   const size_t recv = (size_t)nw * cl * ((Bp + cl - 1) / cl) * kMmaPStride * 4;
-  return mma_stage_bytes(Bp, nw) + recv;
+  return mma_stage_bytes(Bp, nw, kcr) + recv;
 }
 
 template <int NT, bool GU>
@@ -935,7 +938,8 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
                               int bi, int bo, long long dout, cudaStream_t s) {
   constexpr int NW = GU ? 2 : 1;
   const int Bp = (B + 7) & ~7;
-  const size_t smem = mma_smem_bytes(Bp, cl, NW);
+  const int slice = (int)(x.cols / cl);
+  const size_t smem = mma_smem_bytes(Bp, cl, NW, slice < kMmaKc ? slice : kMmaKc);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -943,7 +947,7 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_done & bit)) {
     e = cudaFuncSetAttribute(k_decode_mma<NT, GU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)mma_smem_bytes(GU ? kMmaMaxBGU : kMmaMaxB, 8, NW));
+                             (int)mma_smem_bytes(GU ? kMmaMaxBGU : kMmaMaxB, 8, NW, kMmaKc));
     if (e != cudaSuccess) return e;
     attr_done |= bit;
   }
@@ -962,7 +966,7 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
   return cudaLaunchKernelEx(&cfg, k_decode_mma<NT, GU>, law, q, positions, B,
                             (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr,
                             (const __nv_bfloat16*)(GU ? W2->ptr : W.ptr), W.ld,
-                            (__nv_bfloat16*)y.ptr, y.ld, bi, bo, (int)(x.cols / cl));
+                            (__nv_bfloat16*)y.ptr, y.ld, bi, bo, slice);
 }
 
 static bool aligned16(const aal_mat& m) {
