@@ -47,10 +47,10 @@ NCU_TRAFFIC = {
                         23666944 + 1915136, "aal_tc.cu"),
     ("c2", "down"): ("3e69cfde92c9a578ae451650f886953fad6cc4360be398bc81a3013213bb08d1",
                      40179200 + 2312960, "aal_tc.cu"),
-    ("c2", "decode gate_up B=64"): ("94a41101915e95233a05f199b2fc02bf5c7133c11384046da8c5772b95b74c17",
-                                    4851968, "aal_decode.cu"),
-    ("c2", "decode down B=64"): ("94a41101915e95233a05f199b2fc02bf5c7133c11384046da8c5772b95b74c17",
-                                 2586112, "aal_decode.cu"),
+    ("c2", "decode gate_up B=64"): ("5666616e0a8887abcc355dc9a3026e1f8a01385ef66e4f33975abdff2957c51c",
+                                    4854272, "aal_decode.cu"),
+    ("c2", "decode down B=64"): ("5666616e0a8887abcc355dc9a3026e1f8a01385ef66e4f33975abdff2957c51c",
+                                 2587392, "aal_decode.cu"),
 }
 
 
