@@ -93,11 +93,13 @@ def test_c2_decode_single_type(t):
 
 # Decode shapes around the tensor-core decode kernel's limits: ragged batches,
 # the largest batch it takes (256) and the first it leaves to the SIMT
-# kernels (257), K slices of 16 rows, groups of 16 rows, q up to 32.
+# kernels (257; 1100 reaches the cluster kernel), K slices of 16 rows, groups
+# of 16 rows, q up to 32.
 @pytest.mark.parametrize("law,q,B,din,dout", [
     ("Q2xQ2", 4, 100, 768, 1536),
     ("Q2xQ2", 4, 256, 1536, 768),
     ("Q2xQ2", 4, 257, 768, 1536),
+    ("Q2xQ2", 4, 1100, 768, 1536),
     ("Q", 16, 33, 2048, 1024),
     ("Q", 32, 17, 4096, 2048),
     ("Q", 2, 7, 64, 128),
