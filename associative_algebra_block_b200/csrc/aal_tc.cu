@@ -33,6 +33,10 @@
 // kernel records AAL_ERR_DEVICE_TIMEOUT in the status word, lets in-flight
 // copies and MMAs land, frees TMEM and returns.
 #include <cuda.h>
+
+#include <algorithm>
+#include <queue>
+#include <vector>
 #include <limits.h>
 #include <stdlib.h>
 
@@ -51,6 +55,9 @@ constexpr int kProdWarps = 4;
 constexpr int kSchedWarp = 2 + kEpiWarps + kProdWarps - 1;
 constexpr int kThreads = 32 * (kSchedWarp + 1);
 constexpr int kTileRing = 8;
+// Tile schedules up to this many slots are balanced on the host (longest
+// processing time first onto the least loaded CTA) and passed with the launch.
+constexpr int kMaxOrder = 1024;
 constexpr int kMaxPairs = 256;
 constexpr int kMaxStages = 8;
 constexpr int kSmemBudget = 224 * 1024;  // + 1 KB alignment slack, under the 227 KB per-CTA limit
@@ -125,7 +132,14 @@ struct Params {
   uint16_t pairs[kMaxPairs];
   FastDiv div_n1, div_n3, div_qm1;
   int a_merged, b_merged;  // MN-major operand loaded as one box spanning all its atoms
+  // Schedule: CTA c runs the tiles order[c], order[c + grid], ... up to the
+  // first 0xFFFF (use_order), else tiles c, c + grid, ... below ntiles.
+  int use_order;
+  int nslots;
+  uint16_t order[kMaxOrder];
 };
+
+static_assert(sizeof(Params) <= 4096, "kernel parameters stay within the classic 4 KB limit");
 
 struct TileDesc {
   Seg seg[4];
@@ -509,6 +523,15 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
 
 __device__ __forceinline__ int seg_chunks(const Seg& s) { return (s.len + 63) >> 6; }
 
+// Tile of schedule slot ``slot`` (slot = CTA + round * grid), or -1 when this
+// CTA has no more tiles.
+__device__ __forceinline__ int tile_at(const Params& p, int slot) {
+  if (!p.use_order) return slot < p.ntiles ? slot : -1;
+  if (slot >= p.nslots) return -1;
+  const int t = p.order[slot];
+  return t == 0xFFFF ? -1 : t;
+}
+
 // Copies the description of this role's i-th tile out of the ring and frees
 // the slot (WARP: the whole warp reads it and lane 0 arrives).
 template <bool WARP>
@@ -607,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     const int pw = warp == 0 ? 0 : warp - (1 + kEpiWarps);
     uint32_t it = 0, st = 0, ph = 0, ti = 0;
     bool ok = pw < nprod;
-    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++ti) {
+    for (int ss = tile0; tile_at(p, ss) >= 0 && ok; ss += tstep, ++ti) {
       TileDesc d;
       if (!take_tile<true>(s_tile, tile_full, tile_empty, ti, d, &s_abort)) break;
       for (int s = 0; s < d.nseg && ok; ++s) {
@@ -705,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                                    : ((DUAL == 1 && p.fuse_b) ? p.idesc2 : p.idesc));
       const bool single = PAIR || DUAL == 0 || (DUAL == 1 && p.fuse_b);
       uint64_t so = 0;  // dstage * st
-      for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++tl) {
+      for (int ss = tile0; tile_at(p, ss) >= 0 && ok; ss += tstep, ++tl) {
         TileDesc d;
         if (!take_tile<false>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
         const uint32_t buf = tl & 1u, use = tl >> 1;
@@ -782,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     uint32_t nstore = 0;
     uint32_t tl = 0;
     const int erow = PAIR ? (int)rank * 128 : 0;  // this CTA's 128 rows of the pair's tile
-    for (int tile = tile0; tile < p.ntiles; tile += tstep, ++tl) {
+    for (int ss = tile0; tile_at(p, ss) >= 0; ss += tstep, ++tl) {
       TileDesc d;
       if (!take_tile<true>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
       d.rbase += erow;
@@ -947,7 +970,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     // ------------------------------------------------------ tile decoder
     if (lane == 0) {
       uint32_t i = 0;
-      for (int tile = tile0; tile < p.ntiles; tile += tstep, ++i) {
+      for (int ss = tile0; ; ss += tstep, ++i) {
+        const int tile = tile_at(p, ss);
+        if (tile < 0) break;
         const uint32_t slot = i % kTileRing, ph = (i / kTileRing) & 1u;
         if (!(mbar_try_wait(&tile_empty[slot], ph ^ 1u) ||
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
@@ -1158,6 +1183,71 @@ static void order_pairs(Params& p) {
   }
 }
 
+// Host copy of pair_of (the pair of tile-pair rank ``pr``).
+static void host_pair_of(const Params& p, int pr, int& p0, int& p1) {
+  if (p.npairs_list) {
+    p0 = p.pairs[pr] >> 8;
+    p1 = p.pairs[pr] & 255;
+    return;
+  }
+  const int q = p.q, nd = q * (q - 1);
+  auto diag = [&](int a) {
+    if (p.op == OP_SQUARE || p.op == OP_DW) return a;
+    const int t = a + p.off;
+    return t >= q ? t - q : t;
+  };
+  int r = pr;
+  if (p.diag_first) {
+    if (r < q) { p0 = r; p1 = diag(r); return; }
+    r -= q;
+  } else if (r >= nd) {
+    p0 = r - nd;
+    p1 = diag(p0);
+    return;
+  }
+  p0 = r / (q - 1);
+  const int j = r % (q - 1), dg = diag(p0);
+  p1 = j < dg ? j : j + 1;
+}
+
+// Balances the tiles over ``grid`` CTAs: tiles by decreasing cost (the number
+// of K segments of their table entry; every segment of an op has the same
+// length), each onto the CTA with the least work so far.  Leaves the stride
+// order when the schedule would not fit.
+static void schedule_tiles(Params& p, int grid) {
+  p.use_order = 0;
+  const int nt = p.ntiles;
+  if (grid <= 0 || nt <= grid || nt > kMaxOrder) return;
+  std::vector<int> cost(nt), idx(nt);
+  const int per_pair = p.n1 * p.n3;
+  for (int t = 0; t < nt; ++t) {
+    int p0, p1;
+    host_pair_of(p, t / per_pair, p0, p1);
+    cost[t] = pair_cost(p, p0, p1);
+    idx[t] = t;
+  }
+  std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  std::vector<std::vector<int>> lists(grid);
+  // (load, cta) min-heap
+  std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>,
+                      std::greater<std::pair<long long, int>>> heap;
+  for (int c = 0; c < grid; ++c) heap.push({0, c});
+  for (int t : idx) {
+    auto top = heap.top();
+    heap.pop();
+    lists[top.second].push_back(t);
+    heap.push({top.first + cost[t], top.second});
+  }
+  size_t rounds = 0;
+  for (auto& l : lists) rounds = l.size() > rounds ? l.size() : rounds;
+  if ((long long)rounds * grid > kMaxOrder) return;
+  for (size_t r = 0; r < rounds; ++r)
+    for (int c = 0; c < grid; ++c)
+      p.order[r * grid + c] = r < lists[c].size() ? (uint16_t)lists[c][r] : (uint16_t)0xFFFF;
+  p.nslots = (int)(rounds * grid);
+  p.use_order = 1;
+}
+
 template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false>
 static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (ntiles <= 0) return AAL_OK;
@@ -1182,6 +1272,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   const int sms = num_sms();
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
+    schedule_tiles(p, grid);
     k_tc<A_MN, B_MN, DUAL, false><<<grid, kThreads, smem, s>>>(p);
     note_launch();
     return cuda_status(cudaGetLastError());
