@@ -319,6 +319,27 @@ class ProjFwdBwd:
 
     e2e_step = None
 
+    def oracle_sample(self, rows):
+        """Forward and backward of both projections on an evenly strided row
+        sample (every row type present)."""
+        import oracle
+        rows = min(rows, self.M)
+        sel = np.arange(rows) * (self.M // rows)
+        types = oracle.row_types(self.law, self.q, inputs.packed_positions(self.M, self.seq_len))[sel]
+        data = []
+        for din, dout, seed in ((self.D, self.F, 0), (self.F, self.D, 1)):
+            ins = inputs.projection_inputs(self.M, din, dout, seed=seed, with_dy=True)
+            data.append((ins["X"].f64[sel], ins["W"].f64, ins["dY"].f64[sel]))
+
+        def run():
+            for X, W, dY in data:
+                oracle.project(self.law, self.q, types, X, W)
+                oracle.project_bwd(self.law, self.q, types, X, W, dY)
+
+        return (self.exec_flops * rows) // self.M, run, (
+            f"oracle forward + backward of both projections on {rows} of {self.M} rows "
+            f"(evenly strided, all row types)")
+
 
 class SwigluFwdBwd:
     """Algebraic SwiGLU FFN forward and backward (training step of one FFN):
@@ -405,6 +426,24 @@ class SwigluFwdBwd:
 
     e2e_step = None
 
+    def oracle_sample(self, rows):
+        """SwiGLU forward and backward on an evenly strided row sample."""
+        import oracle
+        rows = min(rows, self.M)
+        sel = np.arange(rows) * (self.M // rows)
+        types = oracle.row_types(self.law, self.q, inputs.packed_positions(self.M, self.seq_len))[sel]
+        ins = inputs.swiglu_inputs(self.D, self.F, self.M, seed=0, dtype="bf16")
+        dY = inputs.Stream(7).normal(self.M, self.D, 1.0, "bf16").f64[sel]
+        X = ins["X"].f64[sel]
+        W = [ins[k].f64 for k in ("Wg", "Wu", "Wd")]
+
+        def run():
+            oracle.swiglu(self.law, self.q, types, X, *W)
+            oracle.swiglu_bwd(self.law, self.q, types, X, *W, dY)
+
+        return (self.exec_flops * rows) // self.M, run, (
+            f"oracle SwiGLU forward + backward on {rows} of {self.M} rows (evenly strided, all row types)")
+
 
 class Square:
     def __init__(self, name, law, q, n):
@@ -443,6 +482,36 @@ class Square:
         torch.matmul(s["X"], s["W"], out=s["Z"])
 
     e2e_step = None
+
+    def oracle_sample(self, rows):
+        """Output blocks (i, k) of the square product, one per 16 requested
+        rows, with the blocks they read drawn from the same distribution
+        (the full 32768^2 operands are not materialised on the host)."""
+        import oracle
+        b = self.n // self.q
+        ntiles = max(1, rows // 16)
+        st = inputs.Stream(7)
+        pairs = [(int(i), int(k)) for i, k in st.integers(ntiles, 2, 0, self.q - 1, "f32").f64]
+        blocks = {}
+
+        def blk(kind, r, c):
+            key = (kind, r, c)
+            if key not in blocks:
+                blocks[key] = st.normal(b, b, self.n ** -0.5, "bf16").f64
+            return blocks[key]
+
+        for i, k in pairs:  # draw the operands before the timed runs
+            for a in oracle.table_entry(self.law, self.q, i, k):
+                blk("X", i, a)
+                blk("W", a, k)
+        flops = sum(2 * b ** 3 * len(oracle.table_entry(self.law, self.q, i, k)) for i, k in pairs)
+
+        def run():
+            for i, k in pairs:
+                oracle.square_tile(self.law, self.q, i, k, lambda r, c: blk("X", r, c),
+                                   lambda r, c: blk("W", r, c))
+
+        return flops, run, f"oracle output blocks of the square product: {ntiles} random (i, k) of {self.q}x{self.q}, b={b}"
 
 
 WORKLOADS = {

@@ -112,3 +112,14 @@ def test_bench_kernel_models_add_up_to_the_step():
     # c4-swiglu: the six timed launches are a subset of the step's work
     w4 = bench.WORKLOADS["c4-swiglu"]()
     assert sum(w4.kernel_model(n, None)[0] for n, _ in w4.timing_slots()) < w4.exec_flops
+
+
+@pytest.mark.parametrize("config", ["c4", "c5", "c4-swiglu"])
+def test_reference_arm_other_workloads(config):
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", config, "--steps", "1", "--warmup", "0", "--ref-rows", "32"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
