@@ -388,7 +388,7 @@ const char* aal_status_string(int32_t status) {
   switch (status) {
     case AAL_OK: return "ok";
     case AAL_ERR_INVALID_ARG: return "invalid argument";
-    case AAL_ERR_UNSUPPORTED: return "unsupported by this build";
+    case AAL_ERR_UNSUPPORTED: return "not supported by the library";
     case AAL_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
     case AAL_ERR_CUDA: return "CUDA runtime error";
     case AAL_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";

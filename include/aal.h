@@ -61,7 +61,7 @@ extern "C" {
 typedef enum aal_status {
   AAL_OK = 0,
   AAL_ERR_INVALID_ARG = 1,    /* bad shape, null pointer, unknown enum value */
-  AAL_ERR_UNSUPPORTED = 2,    /* valid request this build cannot serve      */
+  AAL_ERR_UNSUPPORTED = 2,    /* valid request the library cannot serve      */
   AAL_ERR_ALIGNMENT = 3,      /* pointer / ld misaligned for a required path */
   AAL_ERR_CUDA = 4,           /* a CUDA runtime call failed                  */
   AAL_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out             */
