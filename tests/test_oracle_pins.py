@@ -388,6 +388,46 @@ def test_swiglu_bwd_q1_matches_torch_autograd():
 
 
 @pytest.mark.parametrize("law,q", [("Q2xQ2", 4), ("Q", 3)])
+def test_swiglu_bwd_matches_autograd_of_masked_dense(law, q):
+    # each row type's projection is a dense product with the weight blocks
+    # outside its table row zeroed; torch's float64 autograd through those
+    # masked dense products is an independent derivation of the gradients
+    import torch
+    s = inputs.Stream(120 + q)
+    M, D, F = 3 * q, 2 * q, 4 * q
+    X = s.normal(M, D, 1.0, "f32").f64
+    Wg, Wu = s.normal(D, F, 0.5, "f32").f64, s.normal(D, F, 0.5, "f32").f64
+    Wd = s.normal(F, D, 0.5, "f32").f64
+    dY = s.normal(M, D, 1.0, "f32").f64
+    types = np.arange(M) % q
+    S = oracle.block_table_array(law, q)  # S[t, k, a]
+
+    def mask(t, din, dout):
+        bi, bo = din // q, dout // q
+        m = np.zeros((din, dout))
+        for k in range(q):
+            for a in range(q):
+                if S[t, k, a]:
+                    m[a * bi:(a + 1) * bi, k * bo:(k + 1) * bo] = 1.0
+        return torch.tensor(m)
+
+    t = [torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (X, Wg, Wu, Wd)]
+    rows = []
+    for r in range(M):
+        ty = int(types[r])
+        x = t[0][r:r + 1]
+        g = x @ (t[1] * mask(ty, D, F))
+        u = x @ (t[2] * mask(ty, D, F))
+        h = torch.nn.functional.silu(g) * u
+        rows.append(h @ (t[3] * mask(ty, F, D)))
+    Y = torch.cat(rows)
+    (Y * torch.tensor(dY)).sum().backward()
+    got = oracle.swiglu_bwd(law, q, types, X, Wg, Wu, Wd, dY)
+    for g, ti in zip(got, t):
+        assert np.allclose(g, ti.grad.numpy(), rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("law,q", [("Q2xQ2", 4), ("Q", 3)])
 def test_swiglu_bwd_finite_differences(law, q):
     s = inputs.Stream(100 + q)
     M, D, F = 2 * q, 2 * q, 3 * q
