@@ -180,3 +180,35 @@ def test_plain_c_program_uses_the_boundary(lib, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "table ok" in r.stdout and "counts ok" in r.stdout and "argument check ok" in r.stdout
+
+
+def _declared_arity():
+    """Parameter count of every AAL_API function in include/aal.h."""
+    with open(os.path.join(ROOT, "include", "aal.h")) as f:
+        text = f.read()
+    out = {}
+    for m in re.finditer(r"^AAL_API\s+[\w\s\*]+?\b(aal_\w+)\s*\(([^)]*)\)", text, flags=re.M | re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    # the ctypes declarations of the binding have the header's arity
+    arity = _declared_arity()
+    assert arity, "no declarations parsed"
+    for name, n in arity.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def test_new_entry_points_reject_bad_law_and_q(lib):
+    rule = aal.AalRowTypeRule(0, 16, 0, None)
+    x, Wg, Wd = _m(FAKE, 4, 8), _m(FAKE, 8, 12), _m(FAKE, 12, 8)
+    h, y = _m(FAKE, 4, 12), _m(FAKE, 4, 8)
+    for law, q in ((0, 0), (1, 3), (7, 2)):
+        assert lib.aal_swiglu_decode(law, q, FAKE, x, Wg, Wg, Wd, h, y, None) == aal.AAL_ERR_INVALID_ARG
+        mf, md = _m(FAKE, 16, 12), _m(FAKE, 16, 8)
+        args = [md, Wg, Wg, Wd, mf, md, mf, mf, mf, mf, md, Wg, Wg, Wd]
+        assert lib.aal_swiglu_bwd(law, q, rule, *args, None) == aal.AAL_ERR_INVALID_ARG
