@@ -232,18 +232,28 @@ def test_c4_swiglu():
 
 # ------------------------------------------------- square product Q_256
 def test_c5_square_full_size_sampled_tiles():
+    # Z starts as NaN: a tile the kernel never writes stays non-finite.
+    # Every tile is checked for that on the GPU; against the oracle: all of
+    # tile-row 17, all of tile-column 200, the four corners and 26 random tiles.
     n, q = 32768, 256
     b = n // q
     ins = inputs.square_inputs(n, seed=0, dtype="bf16", want_f64=False)
     X, W = ins["X"].t.cuda(), ins["W"].t.cuda()
-    Z = torch.empty_like(X)
+    Z = torch.full_like(X, float("nan"))
     aal.aal_square_product("Q", q, X, W, Z)
     torch.cuda.synchronize()
     assert aal.aal_last_path() == TENSOR
+    assert aal.aal_get_device_status() == aal.AAL_OK
+    finite = torch.isfinite(Z.view(q, b, q, b)).all(dim=3).all(dim=1)  # [q, q] per tile
+    assert bool(finite.all()), int((~finite).sum())
     Xh, Wh = ins["X"].t, ins["W"].t
     rng = np.random.default_rng(123)
-    tiles = [(0, 0), (0, q - 1), (q - 1, 0), (q - 1, q - 1), (17, 17), (5, 200)]
+    row_i, col_k = 17, 200
+    tiles = [(row_i, k) for k in range(q)] + [(i, col_k) for i in range(q) if i != row_i]
+    tiles += [(0, 0), (0, q - 1), (q - 1, 0), (q - 1, q - 1)]
     tiles += [tuple(int(v) for v in rng.integers(0, q, 2)) for _ in range(26)]
+    Zrow = Z[row_i * b:(row_i + 1) * b].to("cpu", torch.float64).numpy()
+    Zcol = Z[:, col_k * b:(col_k + 1) * b].to("cpu", torch.float64).numpy()
 
     def blk(A, r, c):
         return A[r * b:(r + 1) * b, c * b:(c + 1) * b].to(torch.float64).numpy()
@@ -251,7 +261,12 @@ def test_c5_square_full_size_sampled_tiles():
     worst = 0.0
     for i, k in tiles:
         ref = oracle.square_tile("Q", q, i, k, lambda r, c: blk(Xh, r, c), lambda r, c: blk(Wh, r, c))
-        got = Z[i * b:(i + 1) * b, k * b:(k + 1) * b].to("cpu", torch.float64).numpy()
+        if i == row_i:
+            got = Zrow[:, k * b:(k + 1) * b]
+        elif k == col_k:
+            got = Zcol[i * b:(i + 1) * b]
+        else:
+            got = Z[i * b:(i + 1) * b, k * b:(k + 1) * b].to("cpu", torch.float64).numpy()
         worst = max(worst, oracle.rel_err(got, ref))
     assert worst <= TOL["bf16"], worst
 

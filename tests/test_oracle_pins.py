@@ -483,6 +483,81 @@ def test_swiglu_decode_q1_is_dense_swiglu_and_gate_up_not_symmetric():
 
 
 # --------------------------------------------------------------------------
+# The tile form of the square product (used for large q)
+# --------------------------------------------------------------------------
+
+def _assemble_from_tiles(tile_fn, law, q, X, W):
+    """Z assembled tile by tile from ``tile_fn`` over every output block."""
+    b = X.shape[0] // q
+    Z = np.zeros_like(X)
+
+    def xb(r, c):
+        return X[r * b:(r + 1) * b, c * b:(c + 1) * b]
+
+    def wb(r, c):
+        return W[r * b:(r + 1) * b, c * b:(c + 1) * b]
+
+    for i in range(q):
+        for k in range(q):
+            Z[i * b:(i + 1) * b, k * b:(k + 1) * b] = tile_fn(law, q, i, k, xb, wb)
+    return Z
+
+
+SQUARE_TILE_CASES = [("Q", 2), ("Q", 3), ("Q", 4), ("Q", 5), ("Q2xQ2", 4)]
+
+
+def _square_tile_pin(tile_fn):
+    """The tile form equals the full definition (all q^4 block pairs) exactly
+    on small-integer matrices, and a tile at q = 2 matches the hand-worked
+    entry: Z_01 = X_00 W_01 + X_01 W_11 (source vertex times edge plus edge
+    times target vertex)."""
+    try:
+        for law, q in SQUARE_TILE_CASES:
+            X, W = _int_mats(3 * q, seed=80 + q, count=2)
+            if not np.array_equal(_assemble_from_tiles(tile_fn, law, q, X, W),
+                                  oracle.square_product(law, q, X, W)):
+                return False
+        X, W = _int_mats(6, seed=90, count=2)
+        xb = lambda r, c: X[3 * r:3 * r + 3, 3 * c:3 * c + 3]  # noqa: E731
+        wb = lambda r, c: W[3 * r:3 * r + 3, 3 * c:3 * c + 3]  # noqa: E731
+        by_hand = xb(0, 0) @ wb(0, 1) + xb(0, 1) @ wb(1, 1)
+        if not np.array_equal(tile_fn("Q", 2, 0, 1, xb, wb), by_hand):
+            return False
+        if not np.array_equal(tile_fn("Q", 2, 1, 1, xb, wb), xb(1, 1) @ wb(1, 1)):
+            return False
+    except (ValueError, IndexError, TypeError):
+        return False
+    return True
+
+
+def test_square_tile_equals_square_product_exact():
+    assert _square_tile_pin(oracle.square_tile)
+
+
+def _tile_swapped_x(law, q, i, k, x_block, w_block):
+    return sum(x_block(a, i) @ w_block(a, k) for a in oracle.table_entry(law, q, i, k))
+
+
+def _tile_swapped_w(law, q, i, k, x_block, w_block):
+    return sum(x_block(i, a) @ w_block(k, a) for a in oracle.table_entry(law, q, i, k))
+
+
+def _tile_wrong_chain(law, q, i, k, x_block, w_block):
+    return sum(x_block(i, a) @ w_block(i, k) for a in oracle.table_entry(law, q, i, k))
+
+
+def _tile_first_member_only(law, q, i, k, x_block, w_block):
+    a = oracle.table_entry(law, q, i, k)[0]
+    return x_block(i, a) @ w_block(a, k)
+
+
+@pytest.mark.parametrize("bad", [_tile_swapped_x, _tile_swapped_w, _tile_wrong_chain,
+                                 _tile_first_member_only])
+def test_planted_square_tile_mistakes_are_caught(bad):
+    assert not _square_tile_pin(bad)
+
+
+# --------------------------------------------------------------------------
 # Mutations planted in the oracle: each must trip at least one pin
 # --------------------------------------------------------------------------
 
