@@ -28,6 +28,7 @@ AAL_ERR_ALIGNMENT = 3
 AAL_ERR_CUDA = 4
 AAL_ERR_DEVICE_TIMEOUT = 5
 AAL_ERR_DEVICE_BOUNDS = 6
+AAL_ERR_SCRATCH_LIMIT = 7
 
 LAW = {"Q": 0, "Q2xQ2": 1}
 AAL_BF16, AAL_F32 = 0, 1
@@ -37,7 +38,8 @@ AAL_PATH_AUTO, AAL_PATH_TENSOR, AAL_PATH_GENERAL, AAL_PATH_DECODE = 0, 1, 2, 3
 EXPORTS = ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd", "aal_decode_matvec",
            "aal_swiglu_decode", "aal_swiglu_bwd", "aal_square_product", "aal_block_table", "aal_block_product_count",
            "aal_get_device_status", "aal_status_string", "aal_set_path_policy",
-           "aal_last_path", "aal_launch_count", "aal_version", "aal_set_timing_events")
+           "aal_last_path", "aal_launch_count", "aal_version", "aal_set_timing_events",
+           "aal_swiglu_decode_noalloc")
 AAL_KERNEL_PROJECT, AAL_KERNEL_GATE_UP, AAL_KERNEL_BWD_DX = 1, 2, 3
 AAL_KERNEL_BWD_DW, AAL_KERNEL_SQUARE, AAL_KERNEL_DECODE = 4, 5, 6
 AAL_KERNEL_DECODE_GATE_UP, AAL_KERNEL_SWIGLU_BWD = 7, 8
@@ -81,6 +83,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
             "aal_swiglu_decode": ([i32, i32, vp, AalMat, AalMat, AalMat, AalMat, AalMat, AalMat, vp],
                                   i32),
             "aal_swiglu_bwd": ([i32, i32, AalRowTypeRule] + [AalMat] * 14 + [vp], i32),
+            "aal_swiglu_decode_noalloc": ([i32, i32, vp, AalMat, AalMat, AalMat, AalMat, AalMat, vp],
+                                          i32),
             "aal_project_bwd": ([i32, i32, AalRowTypeRule, AalMat, AalMat, AalMat, AalMat, AalMat,
                                  i32, vp], i32),
             "aal_decode_matvec": ([i32, i32, vp, AalMat, AalMat, AalMat, vp], i32),
@@ -203,6 +207,17 @@ def aal_swiglu_decode(law, q, positions, x, Wg, Wu, Wd, h, y, stream=None):
     _check(load().aal_swiglu_decode(_law(law), q, positions.data_ptr() if positions.numel() else None,
                                     mat(x), mat(Wg), mat(Wu), mat(Wd), mat(h), mat(y), _stream(stream)),
            "aal_swiglu_decode")
+
+
+def aal_swiglu_decode_noalloc(law, q, positions, x, Wg, Wu, Wd, y, stream=None):
+    """aal_swiglu_decode with the activation kept in the library's fixed
+    device array (for callers that cannot allocate device memory)."""
+    if positions.dtype != torch.int64:
+        raise ValueError("positions must be int64")
+    _check(load().aal_swiglu_decode_noalloc(_law(law), q,
+                                            positions.data_ptr() if positions.numel() else None,
+                                            mat(x), mat(Wg), mat(Wu), mat(Wd), mat(y), _stream(stream)),
+           "aal_swiglu_decode_noalloc")
 
 
 def aal_square_product(law, q, X, W, Z, stream=None):

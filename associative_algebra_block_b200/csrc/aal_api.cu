@@ -393,6 +393,7 @@ const char* aal_status_string(int32_t status) {
     case AAL_ERR_CUDA: return "CUDA runtime error";
     case AAL_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
     case AAL_ERR_DEVICE_BOUNDS: return "a kernel met an out-of-range row type or position";
+    case AAL_ERR_SCRATCH_LIMIT: return "request larger than the library's fixed device scratch";
     default: return "unknown status";
   }
 }

@@ -4,3 +4,4 @@
 #include "aal_simt.cu"
 #include "aal_decode.cu"
 #include "aal_tc.cu"
+#include "aal_fixed_scratch.cu"

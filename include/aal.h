@@ -65,7 +65,8 @@ typedef enum aal_status {
   AAL_ERR_ALIGNMENT = 3,      /* pointer / ld misaligned for a required path */
   AAL_ERR_CUDA = 4,           /* a CUDA runtime call failed                  */
   AAL_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out             */
-  AAL_ERR_DEVICE_BOUNDS = 6   /* a kernel met an out-of-range index (type)   */
+  AAL_ERR_DEVICE_BOUNDS = 6,  /* a kernel met an out-of-range index (type)   */
+  AAL_ERR_SCRATCH_LIMIT = 7   /* request larger than a fixed device scratch   */
 } aal_status;
 
 typedef enum aal_law {
@@ -198,6 +199,34 @@ AAL_API aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* posi
 AAL_API aal_status aal_swiglu_decode(int32_t law, int32_t q, const int64_t* positions,
                              aal_mat x, aal_mat Wg, aal_mat Wu, aal_mat Wd, aal_mat h,
                              aal_mat y, void* stream);
+
+/*
+ * aal_swiglu_decode without the caller's activation buffer.  The paper has no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory, for example a plug-in inside a host application that owns
+ * every device allocation through its own pool and forbids direct cudaMalloc,
+ * or a real-time decode loop in which cudaMalloc's implicit device-wide
+ * synchronisation is not allowed.
+ *   Arguments, results and errors are those of aal_swiglu_decode without h:
+ *   positions device int64 [B]; x [B, D]; Wg, Wu [D, F]; Wd [F, D];
+ *   y [B, D] (overwritten).  The activation h [B, F] is kept instead in one
+ *   fixed array of the library's own device memory, 4 MiB on every device
+ *   that loads the library, held until the process exits.
+ * Limit: B * F * (2 for bf16, 4 for fp32) <= 4,194,304 bytes (for example
+ * B <= 1365 at F = 1536 in bf16); a larger request returns
+ * AAL_ERR_SCRATCH_LIMIT before anything is launched.
+ * The call allocates nothing and frees nothing.  Its first call on a device
+ * looks up the array's device address once (cudaGetSymbolAddress with that
+ * device current); make that first call before any stream capture.
+ * Every call shares the one array, which keeps the last call's contents;
+ * nothing in it has to start at zero (each call writes the rows of h it reads
+ * first).  Calls whose work overlaps on the GPU (different streams without
+ * an ordering between them) race on the array and give wrong results: order
+ * them on one stream or with events.
+ */
+AAL_API aal_status aal_swiglu_decode_noalloc(int32_t law, int32_t q, const int64_t* positions,
+                                     aal_mat x, aal_mat Wg, aal_mat Wu, aal_mat Wd,
+                                     aal_mat y, void* stream);
 
 /*
  * Full (not row-typed) product of square block matrices, Z = X * W
