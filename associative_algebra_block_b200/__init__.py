@@ -143,6 +143,41 @@ def mat(t: torch.Tensor | None) -> AalMat:
     return AalMat(t.data_ptr() if t.numel() > 0 else None, dt, rows, cols, max(ld, cols))
 
 
+def _index_vector(t: torch.Tensor, dtype: torch.dtype, n: int, what: str, like: torch.Tensor | None):
+    """Checks an index tensor the kernels read directly: ``dtype``, 1-D,
+    contiguous, exactly ``n`` entries, and (when it has entries) on the CUDA
+    device of ``like``.  A host or short tensor would make a kernel read the
+    wrong memory, so it is refused here."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{what} must be a torch tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}")
+    if t.dim() != 1:
+        raise ValueError(f"{what} must be 1-D")
+    if t.numel() != n:
+        raise ValueError(f"{what} must have {n} entries (has {t.numel()})")
+    if n == 0:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if like is not None and like.numel() > 0 and like.device != t.device:
+        raise ValueError(f"{what} is on {t.device}, the matrices on {like.device}")
+
+
+def _checked_rule(rule, rows: int, like: torch.Tensor | None):
+    """An explicit-type rule's tensor must hold one int32 type per row."""
+    if rule.kind == AAL_TYPES_EXPLICIT:
+        types = getattr(rule, "_types", None)
+        if types is None:
+            if rows > 0:
+                raise ValueError("explicit row types: build the rule with row_rule(types=...)")
+        else:
+            _index_vector(types, torch.int32, rows, "types", like)
+    return rule
+
+
 def row_rule(seq_len: int | None = None, pos_offset: int = 0,
              types: torch.Tensor | None = None) -> AalRowTypeRule:
     """Row-type rule: position-derived (packed sequences of ``seq_len``) or
@@ -174,36 +209,38 @@ def _stream(stream) -> int | None:
 
 
 def aal_project_fwd(law, q, rule, X, W, Y, stream=None):
+    rule = _checked_rule(rule, X.shape[0], X)
     _check(load().aal_project_fwd(_law(law), q, rule, mat(X), mat(W), mat(Y), _stream(stream)),
            "aal_project_fwd")
 
 
 def aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y, stream=None):
+    rule = _checked_rule(rule, X.shape[0], X)
     _check(load().aal_swiglu_fwd(_law(law), q, rule, mat(X), mat(Wg), mat(Wu), mat(Wd), mat(H),
                                  mat(Y), _stream(stream)), "aal_swiglu_fwd")
 
 
 def aal_project_bwd(law, q, rule, X, W, dY, dX=None, dW=None, accumulate_dW=False, stream=None):
+    rule = _checked_rule(rule, X.shape[0], X)
     _check(load().aal_project_bwd(_law(law), q, rule, mat(X), mat(W), mat(dY), mat(dX), mat(dW),
                                   int(bool(accumulate_dW)), _stream(stream)), "aal_project_bwd")
 
 
 def aal_decode_matvec(law, q, positions, x, W, y, stream=None):
-    if positions.dtype != torch.int64:
-        raise ValueError("positions must be int64")
+    _index_vector(positions, torch.int64, x.shape[0], "positions", x)
     _check(load().aal_decode_matvec(_law(law), q, positions.data_ptr() if positions.numel() else None,
                                     mat(x), mat(W), mat(y), _stream(stream)), "aal_decode_matvec")
 
 
 def aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, G, U, dG, dU, dX, dWg, dWu, dWd, stream=None):
+    rule = _checked_rule(rule, X.shape[0], X)
     _check(load().aal_swiglu_bwd(_law(law), q, rule, *(mat(t) for t in (X, Wg, Wu, Wd, H, dY, G, U, dG,
                                                                          dU, dX, dWg, dWu, dWd)),
                                  _stream(stream)), "aal_swiglu_bwd")
 
 
 def aal_swiglu_decode(law, q, positions, x, Wg, Wu, Wd, h, y, stream=None):
-    if positions.dtype != torch.int64:
-        raise ValueError("positions must be int64")
+    _index_vector(positions, torch.int64, x.shape[0], "positions", x)
     _check(load().aal_swiglu_decode(_law(law), q, positions.data_ptr() if positions.numel() else None,
                                     mat(x), mat(Wg), mat(Wu), mat(Wd), mat(h), mat(y), _stream(stream)),
            "aal_swiglu_decode")
@@ -212,8 +249,7 @@ def aal_swiglu_decode(law, q, positions, x, Wg, Wu, Wd, h, y, stream=None):
 def aal_swiglu_decode_noalloc(law, q, positions, x, Wg, Wu, Wd, y, stream=None):
     """aal_swiglu_decode with the activation kept in the library's fixed
     device array (for callers that cannot allocate device memory)."""
-    if positions.dtype != torch.int64:
-        raise ValueError("positions must be int64")
+    _index_vector(positions, torch.int64, x.shape[0], "positions", x)
     _check(load().aal_swiglu_decode_noalloc(_law(law), q,
                                             positions.data_ptr() if positions.numel() else None,
                                             mat(x), mat(Wg), mat(Wu), mat(Wd), mat(y), _stream(stream)),

@@ -265,6 +265,13 @@ AAL_API int64_t aal_block_product_count(int32_t law, int32_t q, int32_t row_type
  * Synchronizes ``stream``, then reads and clears the device status word of
  * the current device: AAL_OK, AAL_ERR_DEVICE_TIMEOUT or
  * AAL_ERR_DEVICE_BOUNDS (or AAL_ERR_CUDA if the synchronization failed).
+ * The word is one per device, shared by every stream and thread: the first
+ * error a kernel records wins until the word is read, and reading clears it.
+ * Only ``stream`` is synchronized, so a kernel still running on another
+ * stream may record an error after the read (it then shows up on a later
+ * read), and one caller's read consumes an error another stream's kernel
+ * recorded.  Synchronize the device, or every stream in use, before reading
+ * when the answer must cover all of them.
  */
 AAL_API aal_status aal_get_device_status(void* stream);
 

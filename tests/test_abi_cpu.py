@@ -148,7 +148,7 @@ def test_empty_inputs_launch_nothing(lib):
 
 def test_status_strings(lib):
     seen = set()
-    for code in range(7):
+    for code in range(8):
         s = aal.aal_status_string(code)
         assert s and s not in seen
         seen.add(s)
@@ -212,3 +212,34 @@ def test_new_entry_points_reject_bad_law_and_q(lib):
         mf, md = _m(FAKE, 16, 12), _m(FAKE, 16, 8)
         args = [md, Wg, Wg, Wd, mf, md, mf, mf, mf, mf, md, Wg, Wg, Wd]
         assert lib.aal_swiglu_bwd(law, q, rule, *args, None) == aal.AAL_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_short_or_strided_index_tensors():
+    # the kernels read positions / explicit types through raw pointers: the
+    # binding refuses anything but a 1-D contiguous device tensor of the
+    # right length and dtype before any call reaches the library
+    import torch
+    x = torch.empty(4, 8, dtype=torch.bfloat16)
+    W = torch.empty(8, 8, dtype=torch.bfloat16)
+    y = torch.empty(4, 8, dtype=torch.bfloat16)
+    cases = [
+        (torch.arange(4), "CUDA device"),              # a host tensor
+        (torch.arange(3), "4 entries"),                # too short
+        (torch.arange(4, dtype=torch.int32), "int64"), # wrong dtype
+        (torch.arange(8).view(2, 4), "1-D"),           # not a vector
+    ]
+    for pos, msg in cases:
+        for call in (lambda p: aal.aal_decode_matvec("Q", 2, p, x, W, y),
+                     lambda p: aal.aal_swiglu_decode("Q", 2, p, x, W, W, W, y, y),
+                     lambda p: aal.aal_swiglu_decode_noalloc("Q", 2, p, x, W, W, W, y)):
+            with pytest.raises(ValueError, match=msg):
+                call(pos)
+    X = torch.empty(6, 8, dtype=torch.bfloat16)
+    Y = torch.empty(6, 8, dtype=torch.bfloat16)
+    for types, msg in ((torch.zeros(6, dtype=torch.int32), "CUDA device"),
+                       (torch.zeros(5, dtype=torch.int32), "6 entries")):
+        rule = aal.row_rule(types=types)
+        with pytest.raises(ValueError, match=msg):
+            aal.aal_project_fwd("Q", 2, rule, X, W, Y)
+        with pytest.raises(ValueError, match=msg):
+            aal.aal_project_bwd("Q", 2, rule, X, W, Y, X, W)

@@ -96,22 +96,53 @@ def test_reference_arm_rank0_prints_one_contract_line():
 
 def test_bench_kernel_models_add_up_to_the_step():
     # the per-launch FLOP models of the c2 step's kernels sum to the step's
-    # executed FLOPs (so a kernel's roofline and the step's value agree)
+    # executed FLOPs (so a kernel's roofline and the step's value agree), and
+    # so do the groups of back-to-back launches
     import torch
     import bench
     from associative_algebra_block_b200 import inputs
     wl = bench.WORKLOADS["c2"]()
     st = inputs.Stream(100)
-    dec = [{"pos": torch.from_numpy(st.positions(B, wl.seq_len))} for B in wl.decode_batches]
+    wl.sets = [{"dec": [{"pos": torch.from_numpy(st.positions(B, wl.seq_len))}
+                        for B in wl.decode_batches]}]
     total = 0
     for name, _ in wl.timing_slots():
-        flops, byts = wl.kernel_model(name, [{"dec": dec}])
+        flops, byts = wl.kernel_model(name)
         assert byts > 0
         total += flops
     assert total == wl.exec_flops
+    assert sum(wl.group_model(g)[0] for g in wl.group_names()) == wl.exec_flops
     # c4-swiglu: the six timed launches are a subset of the step's work
     w4 = bench.WORKLOADS["c4-swiglu"]()
-    assert sum(w4.kernel_model(n, None)[0] for n, _ in w4.timing_slots()) < w4.exec_flops
+    assert sum(w4.kernel_model(n)[0] for n, _ in w4.timing_slots()) < w4.exec_flops
+
+
+@pytest.mark.parametrize("law,q", [("Q", 1), ("Q", 2), ("Q", 5), ("Q", 32), ("Q2xQ2", 4)])
+def test_bench_work_accounting_matches_the_oracle_table(law, q):
+    # the bench counts FLOPs from closed forms (it never loads libaal or the
+    # oracle on the GPU arm); they must agree with the oracle's table
+    import bench
+    import oracle
+    S = oracle.block_table(law, q)
+    for t in range(q):
+        for k in range(q):
+            assert bench._members(law, q, t, k) == tuple(S[t][k])
+    assert bench._per_row(law, q) == oracle.block_product_count(law, q, True)
+    assert bench._square_count(law, q) == oracle.block_product_count(law, q, False)
+
+
+def test_reference_arm_never_loads_libaal():
+    code = ("import sys; sys.argv = ['bench.py', '--impl', 'reference', '--steps', '1', "
+            "'--warmup', '0', '--ref-rows', '16']\n"
+            "import bench\n"
+            "bench.main()\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "print('LIBAAL_MAPPED' if 'libaal' in maps else 'LIBAAL_NOT_MAPPED')\n")
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                       env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip().splitlines()[-1] == "LIBAAL_NOT_MAPPED"
 
 
 @pytest.mark.parametrize("config", ["c4", "c5", "c4-swiglu"])
