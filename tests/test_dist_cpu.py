@@ -154,3 +154,77 @@ def test_reference_arm_other_workloads(config):
     assert r.returncode == 0, r.stderr
     d = json.loads(r.stdout.strip().splitlines()[-1])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _shard_worker(rank, world, port, q_out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import numpy as np
+        import oracle
+        from associative_algebra_block_b200 import inputs
+        from associative_algebra_block_b200.sharding import token_shard
+        law, q, L, M, din, dout = "Q2xQ2", 4, 12, 5 * 12 + 7, 8, 12
+        s = inputs.Stream(70)
+        X = s.integers(M, din, -3, 3, "f32").f64
+        W = s.integers(din, dout, -3, 3, "f32").f64
+        dY = s.integers(M, dout, -3, 3, "f32").f64
+        r0, r1 = token_shard(M, L, world, rank)
+        # the position rule is unchanged on the shard: it starts at a sequence start
+        types = oracle.row_types(law, q, inputs.packed_positions(r1 - r0, L))
+        Y = oracle.project(law, q, types, X[r0:r1], W)
+        dX, dW = oracle.project_bwd(law, q, types, X[r0:r1], W, dY[r0:r1])
+        # forward: no exchange; the rows are gathered here only to check them
+        parts = [None] * world
+        dist.all_gather_object(parts, (r0, r1, Y, dX))
+        # backward: the weight gradient is a sum over tokens -> one all-reduce
+        t = torch.from_numpy(dW.copy())
+        dist.all_reduce(t)
+        q_out.put((rank, parts, t.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_token_shards_reassemble_the_single_rank_result():
+    import numpy as np
+    import oracle
+    from associative_algebra_block_b200 import inputs
+    world = 2
+    ctx = mp.get_context("spawn")
+    q_out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, q_out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q_out.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    law, q, L, M, din, dout = "Q2xQ2", 4, 12, 5 * 12 + 7, 8, 12
+    s = inputs.Stream(70)
+    X = s.integers(M, din, -3, 3, "f32").f64
+    W = s.integers(din, dout, -3, 3, "f32").f64
+    dY = s.integers(M, dout, -3, 3, "f32").f64
+    types = oracle.row_types(law, q, inputs.packed_positions(M, L))
+    Y = oracle.project(law, q, types, X, W)
+    dX, dW = oracle.project_bwd(law, q, types, X, W, dY)
+    for rank, parts, dW_sum in out:
+        covered = sorted((r0, r1) for r0, r1, _, _ in parts)
+        assert covered[0][0] == 0 and covered[-1][1] == M
+        assert all(a[1] == b[0] for a, b in zip(covered, covered[1:]))
+        for r0, r1, Ys, dXs in parts:
+            assert r0 % L == 0  # shards start at a sequence start
+            assert np.array_equal(Ys, Y[r0:r1]) and np.array_equal(dXs, dX[r0:r1])
+        assert np.array_equal(dW_sum, dW)  # exact on small integers
+
+
+@pytest.mark.parametrize("rows,seq_len,world", [(0, 4, 2), (10, 4, 3), (12, 4, 3), (12288, 1536, 8),
+                                                (7, 10, 4)])
+def test_token_shard_covers_rows_by_whole_sequences(rows, seq_len, world):
+    from associative_algebra_block_b200.sharding import token_shard
+    spans = [token_shard(rows, seq_len, world, r) for r in range(world)]
+    assert spans[0][0] == 0 and spans[-1][1] == rows
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 == b0
+    for r0, r1 in spans:
+        assert r0 <= r1 and (r0 % seq_len == 0 or r0 == rows)
