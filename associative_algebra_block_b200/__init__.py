@@ -34,15 +34,16 @@ LAW = {"Q": 0, "Q2xQ2": 1}
 AAL_BF16, AAL_F32 = 0, 1
 AAL_TYPES_POSITION, AAL_TYPES_EXPLICIT = 0, 1
 AAL_PATH_AUTO, AAL_PATH_TENSOR, AAL_PATH_GENERAL, AAL_PATH_DECODE = 0, 1, 2, 3
+AAL_CALL_PROJECT_FWD, AAL_CALL_SWIGLU_FWD = 1, 2
 
 EXPORTS = ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd", "aal_decode_matvec",
            "aal_swiglu_decode", "aal_swiglu_bwd", "aal_square_product", "aal_block_table", "aal_block_product_count",
            "aal_get_device_status", "aal_status_string", "aal_set_path_policy",
            "aal_last_path", "aal_launch_count", "aal_version", "aal_set_timing_events",
-           "aal_swiglu_decode_noalloc")
+           "aal_swiglu_decode_noalloc", "aal_workspace_size", "aal_set_workspace")
 AAL_KERNEL_PROJECT, AAL_KERNEL_GATE_UP, AAL_KERNEL_BWD_DX = 1, 2, 3
 AAL_KERNEL_BWD_DW, AAL_KERNEL_SQUARE, AAL_KERNEL_DECODE = 4, 5, 6
-AAL_KERNEL_DECODE_GATE_UP, AAL_KERNEL_SWIGLU_BWD = 7, 8
+AAL_KERNEL_DECODE_GATE_UP, AAL_KERNEL_SWIGLU_BWD, AAL_KERNEL_FFN_DECODE = 7, 8, 9
 
 
 class AalError(RuntimeError):
@@ -98,6 +99,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
             "aal_launch_count": ([i32], i64),
             "aal_version": ([], i32),
             "aal_set_timing_events": ([i32, vp, vp], i32),
+            "aal_workspace_size": ([i32, i32, i32, AalRowTypeRule, i64, i64, i64], i64),
+            "aal_set_workspace": ([vp, ctypes.c_uint64], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -297,6 +300,32 @@ def aal_set_timing_events(kernel: int, before=None, after=None):
     b = before.cuda_event if before is not None else None
     a = after.cuda_event if after is not None else None
     _check(load().aal_set_timing_events(int(kernel), b, a), "aal_set_timing_events")
+
+
+def aal_workspace_size(call, law, q, rule, rows, d_in, d_hidden=0) -> int:
+    """Bytes of device workspace the call needs for explicit or ragged row
+    types (0: none needed)."""
+    n = int(load().aal_workspace_size(int(call), _law(law), q, rule, int(rows), int(d_in), int(d_hidden)))
+    if n < 0:
+        raise ValueError("aal_workspace_size: invalid arguments")
+    return n
+
+
+_workspace_keep = threading.local()
+
+
+def aal_set_workspace(buf: torch.Tensor | None):
+    """Device workspace (a CUDA tensor, kept alive by the binding until the
+    next call here on this thread) for the following calls of this thread;
+    None removes it."""
+    if buf is None:
+        _check(load().aal_set_workspace(None, 0), "aal_set_workspace")
+        _workspace_keep.t = None
+        return
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check(load().aal_set_workspace(buf.data_ptr(), buf.numel() * buf.element_size()), "aal_set_workspace")
+    _workspace_keep.t = buf
 
 
 def aal_version() -> int:

@@ -6,6 +6,8 @@
 namespace aal {
 
 static thread_local int t_policy = AAL_PATH_AUTO;
+static thread_local void* t_ws = nullptr;        // aal_set_workspace
+static thread_local uint64_t t_ws_bytes = 0;
 static thread_local int t_last_path = 0;
 static thread_local long long t_launches = 0;
 
@@ -104,6 +106,15 @@ aal_status aal_project_fwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_m
   if (X.rows == 0 || Y.cols == 0) return AAL_OK;
   cudaStream_t s = (cudaStream_t)stream;
   RowTypes rt = make_types(rule, q);
+  if (t_policy != AAL_PATH_GENERAL && t_ws && X.dtype == AAL_BF16 && seg_needed(rt, q, X.rows)) {
+    // explicit or ragged types: rows sorted by type into the workspace, then
+    // the tensor-core path in segment mode
+    const aal_status st = timed(AAL_KERNEL_PROJECT, s, [&] {
+      return seg_project_fwd(law, q, rt, X, W, Y, t_ws, t_ws_bytes, s);
+    });
+    if (st == AAL_OK) { note_path(AAL_PATH_TENSOR); return AAL_OK; }
+    if (st != AAL_ERR_UNSUPPORTED) return st;
+  }
   return dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, X.rows, X, W, Y, s); },
                   [&] { return simt_project(law, q, rt, X, W, Y, s); });
 }
@@ -126,6 +137,13 @@ aal_status aal_swiglu_fwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_ma
   if (M == 0 || D == 0) return AAL_OK;
   cudaStream_t s = (cudaStream_t)stream;
   RowTypes rt = make_types(rule, q);
+  if (t_policy != AAL_PATH_GENERAL && t_ws && dt == AAL_BF16 && seg_needed(rt, q, M)) {
+    const aal_status st = timed(AAL_KERNEL_GATE_UP, s, [&] {
+      return seg_swiglu_fwd(law, q, rt, X, Wg, Wu, Wd, H, Y, t_ws, t_ws_bytes, s);
+    });
+    if (st == AAL_OK) { note_path(AAL_PATH_TENSOR); return AAL_OK; }
+    if (st != AAL_ERR_UNSUPPORTED) return st;
+  }
   int path_gu = 0;
   aal_status st = dispatch(AAL_KERNEL_GATE_UP, s, [&] { return tc_swiglu_gate_up(law, q, rt, M, X, Wg, Wu, H, s); },
                            [&] { return simt_swiglu_gate_up(law, q, rt, X, Wg, Wu, H, s); });
@@ -294,6 +312,13 @@ aal_status aal_swiglu_decode(int32_t law, int32_t q, const int64_t* positions, a
   note_path(0);
   if (B == 0 || D == 0 || F == 0) return AAL_OK;
   cudaStream_t s = (cudaStream_t)stream;
+  if (t_policy != AAL_PATH_GENERAL && ffn_decode_fused_ok(law, q, x, Wg, Wu, Wd, h, y)) {
+    const aal_status fs = timed(AAL_KERNEL_FFN_DECODE, s, [&] {
+      return ffn_decode_fused(law, q, positions, x, Wg, Wu, Wd, h, y, s);
+    });
+    if (fs == AAL_OK) note_path(AAL_PATH_DECODE);
+    return fs;
+  }
   int path = AAL_PATH_DECODE;
   aal_status st = AAL_OK;
   bool handled = false;
@@ -318,7 +343,12 @@ aal_status aal_swiglu_decode(int32_t law, int32_t q, const int64_t* positions, a
   }
   handled = false;
   if (t_policy != AAL_PATH_GENERAL) {
-    st = timed(AAL_KERNEL_DECODE, s, [&] { return decode_matvec(law, q, positions, h, Wd, y, s, &handled); });
+    // up to 16 entries the down decode starts while the gate/up kernel runs
+    // and waits for h on the device (programmatic dependent launch; measured
+    // on B200: 9.2 -> 8.4 us per FFN step at one entry, slower at 64)
+    st = timed(AAL_KERNEL_DECODE, s, [&] {
+      return decode_matvec(law, q, positions, h, Wd, y, s, &handled, path == AAL_PATH_DECODE && B <= 16);
+    });
     if (st != AAL_OK) return st;
   }
   if (!handled) {
@@ -399,9 +429,25 @@ const char* aal_status_string(int32_t status) {
 }
 
 aal_status aal_set_timing_events(int32_t kernel, void* before, void* after) {
-  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_SWIGLU_BWD) return AAL_ERR_INVALID_ARG;
+  if (kernel < AAL_KERNEL_PROJECT || kernel > AAL_KERNEL_FFN_DECODE) return AAL_ERR_INVALID_ARG;
   t_ev_before[kernel] = (cudaEvent_t)before;
   t_ev_after[kernel] = (cudaEvent_t)after;
+  return AAL_OK;
+}
+
+int64_t aal_workspace_size(int32_t call, int32_t law, int32_t q, aal_row_type_rule rule, int64_t rows,
+                           int64_t d_in, int64_t d_hidden) {
+  if (!valid_law(law, q) || rows < 0 || d_in < 0 || d_hidden < 0 || !valid_rule(rule, rows)) return -1;
+  if (call != AAL_CALL_PROJECT_FWD && call != AAL_CALL_SWIGLU_FWD) return -1;
+  const RowTypes rt = make_types(rule, q);
+  if (rows == 0 || !seg_needed(rt, q, rows)) return 0;
+  return seg_workspace_bytes(q, rows, d_in, call == AAL_CALL_SWIGLU_FWD ? d_hidden : 0);
+}
+
+aal_status aal_set_workspace(void* device_ptr, uint64_t bytes) {
+  if (device_ptr && ((uintptr_t)device_ptr % 256) != 0) return AAL_ERR_ALIGNMENT;
+  t_ws = bytes ? device_ptr : nullptr;
+  t_ws_bytes = device_ptr ? bytes : 0;
   return AAL_OK;
 }
 

@@ -726,6 +726,9 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   __shared__ unsigned s_pres[8][2];
   __shared__ unsigned char s_used[64];  // groups of the CTA's K slice that some entry uses
   cg::cluster_group cluster = cg::this_cluster();
+  // a launch that depends on this one (programmatic stream serialization)
+  // may start now: it only prefetches its weights before waiting for us
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // every CTA of the cluster is running before any writes into a peer
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
@@ -750,7 +753,7 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   long long my_pos = -1;
   if (tid < B) my_pos = pos[tid];
 
-  auto stage = [&](int r0, int rows, bool all_rows) {
+  auto stage_w = [&](int r0, int rows, bool all_rows) {
     for (int i = tid; i < rows * 8; i += blockDim.x) {
       const int r = i >> 3, ch = i & 7;
       if (all_rows || s_used[(r0 + r) / bi - g0]) {
@@ -761,6 +764,8 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
                      W2 + (long long)(r0 + r) * ldw + c0 + ch * 8, 16);
       }
     }
+  };
+  auto stage_x = [&](int r0, int rows) {
     // item i = n * xch + ch, walked without a division per item
     const int xch = rows >> 3, dq = 256 / xch, dr = 256 - dq * xch;
     int n = tid / xch, ch = tid - n * xch;
@@ -773,8 +778,15 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  // round 0's copies go out first
-  stage(ks0, kcr, true);
+  // round 0's copies go out first.  When this launch depends on the previous
+  // one (the down projection of an FFN decode step, launched with
+  // programmatic stream serialization while the gate/up kernel still runs),
+  // only the weights are fetched before griddepcontrol.wait: the activations
+  // are that kernel's output.  Without such a dependency the wait returns at
+  // once.
+  stage_w(ks0, kcr, true);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  stage_x(ks0, kcr);
 
   // 1. row type of every entry (-1 for padding and invalid positions) and
   //    the set of types present
@@ -823,7 +835,10 @@ k_decode_mma(int law, int q, const int64_t* __restrict__ pos, int B,
   for (int kc = 0; kc < slice; kc += kcr) {
     const int rows = min(kcr, slice - kc);
     const int r0 = ks0 + kc;  // first weight row of this round
-    if (kc > 0) stage(r0, rows, false);
+    if (kc > 0) {
+      stage_w(r0, rows, false);
+      stage_x(r0, rows);
+    }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();
     // 3. MMAs over the used 16-row steps; an entry whose table row does not
@@ -935,7 +950,7 @@ static size_t mma_smem_bytes(int Bp, int cl, int nw, int kcr) {
 template <int NT, bool GU>
 static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, int B,
                               const aal_mat& x, const aal_mat& W, const aal_mat* W2, const aal_mat& y,
-                              int bi, int bo, long long dout, cudaStream_t s) {
+                              int bi, int bo, long long dout, cudaStream_t s, bool pdl = false) {
   constexpr int NW = GU ? 2 : 1;
   const int Bp = (B + 7) & ~7;
   const int slice = (int)(x.cols / cl);
@@ -956,13 +971,15 @@ static cudaError_t launch_mma(int cl, int law, int q, const int64_t* positions, 
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = cl;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_decode_mma<NT, GU>, law, q, positions, B,
                             (const __nv_bfloat16*)x.ptr, x.ld, (const __nv_bfloat16*)W.ptr,
                             (const __nv_bfloat16*)(GU ? W2->ptr : W.ptr), W.ld,
@@ -1028,7 +1045,7 @@ aal_status decode_gate_up(int law, int q, const int64_t* positions, const aal_ma
 }
 
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
-                         const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled) {
+                         const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled, bool pdl) {
   *handled = true;
   const long long B = x.rows, dout = W.cols;
   if (B == 0 || dout == 0) return AAL_OK;
@@ -1044,9 +1061,9 @@ aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat
     int cl = 8;
     while (cl > 1 && (x.cols % (16 * cl)) != 0) cl >>= 1;
     cudaError_t e;
-    if (B <= 16) e = launch_mma<1, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
-    else if (B <= 64) e = launch_mma<4, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
-    else e = launch_mma<16, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s);
+    if (B <= 16) e = launch_mma<1, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s, pdl);
+    else if (B <= 64) e = launch_mma<4, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s, pdl);
+    else e = launch_mma<16, false>(cl, law, q, positions, (int)B, x, W, nullptr, y, bi, bo, dout, s, pdl);
     note_launch();
     return cuda_status(e);
   }

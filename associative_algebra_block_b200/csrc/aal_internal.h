@@ -92,8 +92,17 @@ aal_status simt_square(int law, int q, const aal_mat& X, const aal_mat& W, const
 aal_status decode_gate_up(int law, int q, const int64_t* positions, const aal_mat& x,
                           const aal_mat& Wg, const aal_mat& Wu, const aal_mat& h, cudaStream_t s,
                           bool* handled);
+// pdl: launch with programmatic stream serialization (the kernel fetches its
+// weights while the previous launch on the stream finishes).
 aal_status decode_matvec(int law, int q, const int64_t* positions, const aal_mat& x,
-                         const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled);
+                         const aal_mat& W, const aal_mat& y, cudaStream_t s, bool* handled,
+                         bool pdl = false);
+// One-launch FFN decode step (gate/up/SiLU and down in one kernel).
+bool ffn_decode_fused_ok(int law, int q, const aal_mat& x, const aal_mat& Wg, const aal_mat& Wu,
+                         const aal_mat& Wd, const aal_mat& h, const aal_mat& y);
+aal_status ffn_decode_fused(int law, int q, const int64_t* positions, const aal_mat& x,
+                            const aal_mat& Wg, const aal_mat& Wu, const aal_mat& Wd, const aal_mat& h,
+                            const aal_mat& y, cudaStream_t s);
 
 // ------------------------------------------------------------ tensor-core path
 // Each returns AAL_ERR_UNSUPPORTED (launching nothing) when the shape is not
@@ -111,6 +120,18 @@ aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows,
                              const aal_mat& dY, const aal_mat& dW, int accumulate, cudaStream_t s);
 aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const aal_mat& Z,
                      cudaStream_t s);
+aal_status tc_project_seg(int law, int q, long long rows, const aal_mat& Xg, const aal_mat& Wg,
+                          const aal_mat* Wu, const aal_mat& Y, const int4* tiles, const int* count,
+                          const int* perm, int tmax, const aal_mat* copy, cudaStream_t s);
+
+// ------------------------------------------- explicit / ragged row types
+bool seg_needed(const RowTypes& rt, int q, long long rows);
+int64_t seg_workspace_bytes(int q, long long rows, long long w1, long long w2);
+aal_status seg_project_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& W,
+                           const aal_mat& Y, void* ws, uint64_t ws_bytes, cudaStream_t s);
+aal_status seg_swiglu_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& Wg,
+                          const aal_mat& Wu, const aal_mat& Wd, const aal_mat& H, const aal_mat& Y, void* ws,
+                          uint64_t ws_bytes, cudaStream_t s);
 
 inline aal_status cuda_status(cudaError_t e) { return e == cudaSuccess ? AAL_OK : AAL_ERR_CUDA; }
 

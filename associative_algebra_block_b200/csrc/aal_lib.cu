@@ -4,4 +4,6 @@
 #include "aal_simt.cu"
 #include "aal_decode.cu"
 #include "aal_tc.cu"
+#include "aal_ffn_decode.cu"
+#include "aal_segments.cu"
 #include "aal_fixed_scratch.cu"

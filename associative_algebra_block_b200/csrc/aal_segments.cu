@@ -1,0 +1,220 @@
+// Explicit and ragged row types on the tensor-core path.
+//
+// The strided tensor-core path reads the rows of one type through a TMA view
+// that needs every sequence to be a whole number of q positions long.  When
+// the types are explicit, or the positions do not line up (agihunt.info
+// digest, Transformer-mapping paragraph: a token's type comes from its
+// absolute position, so any packing of sequences is legal), the rows are
+// first sorted by type on the device into a caller workspace: a per-block
+// histogram, one scan that also writes the tcgen05 kernel's tile table (a
+// type's rows in tiles of 128), and a scatter that records the permutation
+// and copies each row of X into its type's contiguous segment.  The tcgen05
+// kernel then runs in segment mode and its epilogue writes every output row
+// back to its original place.  No host synchronisation: the tile count stays
+// on the device and tiles past it are empty.
+#include "aal_internal.h"
+
+namespace aal {
+namespace seg {
+
+constexpr int kThreads = 256;
+constexpr int kRowsPerBlock = 1024;
+constexpr int kMaxQ = 256;
+
+struct Layout {
+  size_t blk, counts, tiles, perm, xg, hg, total;
+  long long G;  // row blocks of the histogram and scatter kernels
+  int tmax;     // bound on the tile table's length
+};
+
+static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Workspace of a call over ``rows`` rows gathering w1 columns (and w2 more
+// for a SwiGLU's hidden activation).
+static Layout layout(int q, long long rows, long long w1, long long w2) {
+  Layout L;
+  L.G = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
+  L.tmax = (int)((rows + 127) / 128 + q);
+  size_t off = 0;
+  L.blk = off;
+  off = up256(off + (size_t)L.G * q * 4);
+  L.counts = off;
+  off = up256(off + (size_t)(q + 4) * 4);
+  L.tiles = off;
+  off = up256(off + (size_t)L.tmax * 16);
+  L.perm = off;
+  off = up256(off + (size_t)rows * 4);
+  L.xg = off;
+  off = up256(off + (size_t)rows * w1 * 2);
+  L.hg = off;
+  off = up256(off + (size_t)rows * w2 * 2);
+  L.total = off;
+  return L;
+}
+
+// 1. per-block histogram of the row types (rows with an invalid type are
+//    left out; row_type records the bounds error)
+__global__ void __launch_bounds__(kThreads) k_seg_hist(RowTypes rt, long long rows, int q, int* blk) {
+  __shared__ int c[kMaxQ];
+  for (int i = threadIdx.x; i < q; i += kThreads) c[i] = 0;
+  __syncthreads();
+  const long long r0 = (long long)blockIdx.x * kRowsPerBlock;
+  for (int i = threadIdx.x; i < kRowsPerBlock && r0 + i < rows; i += kThreads) {
+    const int t = row_type(rt, r0 + i);
+    if (t >= 0) atomicAdd(&c[t], 1);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < q; i += kThreads) blk[(long long)blockIdx.x * q + i] = c[i];
+}
+
+// 2. one block: type totals, segment starts, per-(block, type) scatter
+//    offsets (in place of the histogram), and the tile table
+__global__ void __launch_bounds__(kThreads) k_seg_scan(long long G, int q, int* blk, int* counts,
+                                                       int4* tiles) {
+  __shared__ int tot[kMaxQ];
+  __shared__ int seg[kMaxQ + 1];
+  __shared__ int tst[kMaxQ + 1];
+  for (int t = threadIdx.x; t < q; t += kThreads) {
+    int s = 0;
+    for (long long b = 0; b < G; ++b) s += blk[b * q + t];
+    tot[t] = s;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    seg[0] = 0;
+    tst[0] = 0;
+    for (int t = 0; t < q; ++t) {
+      seg[t + 1] = seg[t] + tot[t];
+      tst[t + 1] = tst[t] + (tot[t] + 127) / 128;
+    }
+    counts[q] = tst[q];  // the tile count the tcgen05 kernel reads
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < q; t += kThreads) {
+    int run = seg[t];
+    for (long long b = 0; b < G; ++b) {
+      const int c = blk[b * q + t];
+      blk[b * q + t] = run;
+      run += c;
+    }
+    counts[t] = tot[t];
+    const int nt = (tot[t] + 127) / 128;
+    for (int i = 0; i < nt; ++i) tiles[tst[t] + i] = make_int4(t, seg[t] + 128 * i, seg[t] + tot[t], 0);
+  }
+}
+
+// 3. each row takes the next place of its type's segment: the permutation
+//    records it and the row of X is copied there (16-byte vectors, one warp
+//    per row)
+__global__ void __launch_bounds__(kThreads) k_seg_scatter(RowTypes rt, long long rows, int q, const int* blk,
+                                                          int* perm, const __nv_bfloat16* X, long long ldx,
+                                                          int cols, __nv_bfloat16* Xg, long long ldg) {
+  __shared__ int cur[kMaxQ];
+  __shared__ int dst[kRowsPerBlock];
+  for (int i = threadIdx.x; i < q; i += kThreads) cur[i] = blk[(long long)blockIdx.x * q + i];
+  __syncthreads();
+  const long long r0 = (long long)blockIdx.x * kRowsPerBlock;
+  const int nr = (int)(rows - r0 < kRowsPerBlock ? rows - r0 : kRowsPerBlock);
+  for (int i = threadIdx.x; i < nr; i += kThreads) {
+    const int t = row_type(rt, r0 + i);
+    const int d = t >= 0 ? atomicAdd(&cur[t], 1) : -1;
+    dst[i] = d;
+    if (d >= 0) perm[d] = (int)(r0 + i);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nv = cols >> 3;
+  for (int i = warp; i < nr; i += kThreads / 32) {
+    const int d = dst[i];
+    if (d < 0) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(X + (r0 + i) * ldx);
+    uint4* out = reinterpret_cast<uint4*>(Xg + (long long)d * ldg);
+    for (int v = lane; v < nv; v += 32) out[v] = src[v];
+  }
+}
+
+static bool rows16(const aal_mat& m) {
+  return m.dtype == AAL_BF16 && ((uintptr_t)m.ptr % 16) == 0 && m.ld % 8 == 0;
+}
+
+}  // namespace seg
+
+// Whether the rows of this rule need the sorted (segment) path: explicit
+// types, or sequences / rows that are not whole multiples of q.
+bool seg_needed(const RowTypes& rt, int q, long long rows) {
+  return !(rt.kind == kTypesPosition && rt.seq_len % q == 0 && rows % q == 0);
+}
+
+int64_t seg_workspace_bytes(int q, long long rows, long long w1, long long w2) {
+  return (int64_t)seg::layout(q, rows, w1, w2).total;
+}
+
+// Sorts the rows by type and gathers X into the workspace's segments.
+static aal_status seg_prepare(int q, const RowTypes& rt, long long rows, const aal_mat& X, char* ws,
+                              const seg::Layout& L, cudaStream_t s) {
+  using namespace seg;
+  int* blk = (int*)(ws + L.blk);
+  int* counts = (int*)(ws + L.counts);
+  int4* tiles = (int4*)(ws + L.tiles);
+  int* perm = (int*)(ws + L.perm);
+  __nv_bfloat16* Xg = (__nv_bfloat16*)(ws + L.xg);
+  k_seg_hist<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk);
+  k_seg_scan<<<1, seg::kThreads, 0, s>>>(L.G, q, blk, counts, tiles);
+  k_seg_scatter<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk, perm, (const __nv_bfloat16*)X.ptr,
+                                                   X.ld, (int)X.cols, Xg, X.cols);
+  note_launch(3);
+  return cuda_status(cudaGetLastError());
+}
+
+// Common eligibility of the segment path (before anything is launched).
+static bool seg_ok(int q, long long rows, const aal_mat& X, const aal_mat* const* mats, int nmats,
+                   void* ws, uint64_t ws_bytes, long long w2) {
+  if (q > seg::kMaxQ || rows <= 0 || rows > (1LL << 30) || !ws || ((uintptr_t)ws % 256) != 0) return false;
+  if (!seg::rows16(X) || (X.cols % 16)) return false;
+  for (int i = 0; i < nmats; ++i)
+    if (!seg::rows16(*mats[i])) return false;
+  return (uint64_t)seg_workspace_bytes(q, rows, X.cols, w2) <= ws_bytes;
+}
+
+aal_status seg_project_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& W,
+                           const aal_mat& Y, void* ws, uint64_t ws_bytes, cudaStream_t s) {
+  const aal_mat* mats[] = {&W, &Y};
+  if (!seg_ok(q, X.rows, X, mats, 2, ws, ws_bytes, 0)) return AAL_ERR_UNSUPPORTED;
+  if ((X.cols / q) % 16 || (W.cols / q) % 16) return AAL_ERR_UNSUPPORTED;
+  const seg::Layout L = seg::layout(q, X.rows, X.cols, 0);
+  char* w = (char*)ws;
+  aal_status st = seg_prepare(q, rt, X.rows, X, w, L, s);
+  if (st != AAL_OK) return st;
+  aal_mat Xg = X;
+  Xg.ptr = w + L.xg;
+  Xg.ld = X.cols;
+  return tc_project_seg(law, q, X.rows, Xg, W, nullptr, Y, (const int4*)(w + L.tiles),
+                        (const int*)(w + L.counts) + q, (const int*)(w + L.perm), L.tmax, nullptr, s);
+}
+
+aal_status seg_swiglu_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& Wg,
+                          const aal_mat& Wu, const aal_mat& Wd, const aal_mat& H, const aal_mat& Y, void* ws,
+                          uint64_t ws_bytes, cudaStream_t s) {
+  const aal_mat* mats[] = {&Wg, &Wu, &Wd, &H, &Y};
+  const long long F = Wg.cols;
+  if (!seg_ok(q, X.rows, X, mats, 5, ws, ws_bytes, F)) return AAL_ERR_UNSUPPORTED;
+  if ((X.cols / q) % 16 || (F / q) % 16) return AAL_ERR_UNSUPPORTED;
+  const seg::Layout L = seg::layout(q, X.rows, X.cols, F);
+  char* w = (char*)ws;
+  aal_status st = seg_prepare(q, rt, X.rows, X, w, L, s);
+  if (st != AAL_OK) return st;
+  aal_mat Xg = X, Hg = H;
+  Xg.ptr = w + L.xg;
+  Xg.ld = X.cols;
+  Hg.ptr = w + L.hg;
+  Hg.ld = F;
+  const int4* tiles = (const int4*)(w + L.tiles);
+  const int* count = (const int*)(w + L.counts) + q;
+  const int* perm = (const int*)(w + L.perm);
+  // gate/up with SiLU*mul: H in the caller's row order, and the gathered
+  // copy the down projection reads
+  st = tc_project_seg(law, q, X.rows, Xg, Wg, &Wu, H, tiles, count, perm, L.tmax, &Hg, s);
+  if (st != AAL_OK) return st;
+  return tc_project_seg(law, q, X.rows, Hg, Wd, nullptr, Y, tiles, count, perm, L.tmax, nullptr, s);
+}
+
+}  // namespace aal

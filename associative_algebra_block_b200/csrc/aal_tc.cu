@@ -63,6 +63,8 @@ constexpr int kMaxStages = 8;
 constexpr int kSmemBudget = 224 * 1024;  // + 1 KB alignment slack, under the 227 KB per-CTA limit
 constexpr int kEpiSmem = kEpiWarps * 2048;  // TMA-store staging
 constexpr unsigned long long kWaitNs = 2000000000ull;
+// Limit of the test stall (see Params::test_stall).
+constexpr unsigned long long kStallNs = 50000000ull;
 
 enum Op : int { OP_FWD = 0, OP_SWIGLU = 1, OP_DX = 2, OP_DW = 3, OP_SQUARE = 4 };
 
@@ -136,6 +138,23 @@ struct Params {
   // first 0xFFFF (use_order), else tiles c, c + grid, ... below ntiles.
   int use_order;
   int nslots;
+  // Test hook: 1 makes the MMA thread first wait on a barrier nothing ever
+  // arrives on, so the bounded wait runs out (after kStallNs), the kernel
+  // records AAL_ERR_DEVICE_TIMEOUT and takes its abort path.
+  int test_stall;
+  // Segment mode (forward ops with explicit or ragged row types): the rows
+  // were gathered type by type into contiguous segments; tile j of the device
+  // table seg_tiles (j < *seg_count) is {type, first row, end of its type's
+  // segment, 0}; tile index = (j * q + k) * n3 + i3.  Output row x of the
+  // gathered order is row seg_perm[x] of the caller's output; with seg_copy
+  // the tile is also written, in the gathered order, to seg_copy.
+  int seg_mode;
+  const int4* seg_tiles;
+  const int* seg_count;
+  const int* seg_perm;
+  __nv_bfloat16* seg_copy;
+  long long ld_copy;
+  FastDiv div_qn3;
   uint16_t order[kMaxOrder];
 };
 
@@ -185,13 +204,14 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity
 }
 // Bounded wait by one thread.  Returns false if the kernel was aborted or the
 // wait ran out (which records the timeout and aborts the kernel).
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                       unsigned long long limit_ns = kWaitNs) {
   const unsigned long long t0 = gtime();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 255u) {
       if (*abort) return false;
-      if (gtime() - t0 > kWaitNs) {
+      if (gtime() - t0 > limit_ns) {
         flag_device_error(kDevTimeout);
         *abort = 1;
         return false;
@@ -461,8 +481,38 @@ __device__ __forceinline__ void pair_of(const Params& p, int pr, int& p0, int& p
   p1 = j < dg ? j : j + 1;
 }
 
+// Segment mode: tile = (j * q + k) * n3 + i3 over the device tile table.
+__device__ __forceinline__ void describe_seg(const Params& p, int tile, TileDesc& d) {
+  const int j = (int)fdiv((uint32_t)tile, p.div_qn3);
+  const int rem = tile - j * p.q * p.n3;
+  const int k = (int)fdiv((uint32_t)rem, p.div_n3);
+  const int i3 = rem - k * p.n3;
+  d.nseg = 0;
+  d.rstride = 1;
+  d.roff = 0;
+  d.a_c1 = 0;
+  d.b_c1 = 0;
+  d.b_f = k * p.bo + i3 * p.wn;
+  d.cbase = d.b_f;
+  if (j >= *(volatile const int*)p.seg_count) {  // past the table: an empty tile
+    d.a_f = 0;
+    d.rbase = 0;
+    d.rlimit = 0;
+    return;
+  }
+  const int4 e = p.seg_tiles[j];
+  add_members(p, d, e.x, k, p.bi, 0);
+  d.a_f = e.y;
+  d.rbase = e.y;
+  d.rlimit = e.z;
+}
+
 // tile = (pair_rank * n1 + i1) * n3 + i3; the pair is (i0, i2) of the op.
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
+  if (p.seg_mode) {
+    describe_seg(p, tile, d);
+    return;
+  }
   const int t3 = (int)fdiv((uint32_t)tile, p.div_n3);
   const int i3 = tile - t3 * p.n3;
   const int pr = (int)fdiv((uint32_t)t3, p.div_n1);
@@ -573,6 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   __shared__ TileDesc s_tile[kTileRing];
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
+  __shared__ int s_last_chunk[kMaxStages];  // last K chunk issued into each stage (-1: none)
+  __shared__ __align__(8) uint64_t stall_bar;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t smem0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -590,6 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       mbar_init(&tempty_bar[b], (PAIR ? 2 : 1) * kEpiWarps);
     }
     mbar_init(&done_bar, 1);
+    mbar_init(&stall_bar, 1);
+    for (int s = 0; s < kMaxStages; ++s) s_last_chunk[s] = -1;
     // a ring slot is free again once every consuming warp has copied it: the
     // producer warps in use, the MMA thread (where this CTA issues) and the
     // epilogue warps
@@ -646,6 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const int kofs = sg.k0 + kc * 64;
             const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
             if (lane == 0 && issuer) mbar_expect_tx(&full_bar[st], (PAIR ? 2u : 1u) * p.stage_bytes);
+            if (lane == 0) atomicMax(&s_last_chunk[st], (int)it);
             const int na = DUAL == 2 ? 2 : 1;
             const int nb = (DUAL == 1 && !PAIR) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
@@ -697,14 +752,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
         }
       }
     }
-    // let every copy this CTA issued land before the CTA can exit (for a pair
-    // the pair's first CTA sees both halves on its own barriers); warp 0 counts
-    // every chunk, so it waits for the last use of each stage
+    // Let every copy this CTA issued land before the CTA can exit (for a pair
+    // the pair's first CTA sees both halves on its own barriers).  The chunks
+    // issued into a stage always form a prefix of that stage's phases: chunk
+    // i + S can only be issued after chunk i was consumed, so on the abort
+    // path a chunk that was never issued stops its stage for good.  Waiting
+    // for the phase of the last chunk actually issued into each stage (across
+    // the four producer warps) therefore covers every copy in flight, on the
+    // normal path and after an abort alike.
+    __syncwarp();
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kProdWarps) : "memory");
     if (warp == 0 && lane == 0 && issuer) {
       for (int st = 0; st < S; ++st) {
-        if ((uint32_t)st >= it) break;
-        const uint32_t last = st + ((it - 1 - st) / S) * S;
-        mbar_wait_teardown(&full_bar[st], (last / S) & 1u);
+        const int last = s_last_chunk[st];
+        if (last >= 0) mbar_wait_teardown(&full_bar[st], ((uint32_t)last / (uint32_t)S) & 1u);
       }
     }
     __syncwarp();
@@ -728,6 +789,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                                    : ((DUAL == 1 && p.fuse_b) ? p.idesc2 : p.idesc));
       const bool single = PAIR || DUAL == 0 || (DUAL == 1 && p.fuse_b);
       uint64_t so = 0;  // dstage * st
+      // test hook: a wait nothing ends, bounded by kStallNs; it records the
+      // timeout and aborts the kernel before the first MMA
+      if (p.test_stall && !mbar_wait(&stall_bar, 0, &s_abort, kStallNs)) ok = false;
       for (int ss = tile0; tile_at(p, ss) >= 0 && ok; ss += tstep, ++tl) {
         TileDesc d;
         if (!take_tile<false>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
@@ -921,7 +985,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             reinterpret_cast<uint4*>(p.out2 + off)[0] = w[0];
             reinterpret_cast<uint4*>(p.out2 + off)[1] = w[1];
           } else if (x < d.rlimit) {
-            __nv_bfloat16* dst = p.out + (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
+            const long long xo = p.seg_mode ? (long long)p.seg_perm[x] : x * d.rstride + d.roff;
+            __nv_bfloat16* dst = p.out + xo * p.ldo + d.cbase + c0;
             if (p.accumulate) {
               uint4 o0 = reinterpret_cast<const uint4*>(dst)[0];
               uint4 o1 = reinterpret_cast<const uint4*>(dst)[1];
@@ -939,6 +1004,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             for (int j = 0; j < 8; ++j) h[j] = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
             reinterpret_cast<uint4*>(dst)[0] = w[0];
             reinterpret_cast<uint4*>(dst)[1] = w[1];
+            if (p.seg_copy) {
+              uint4* cp = reinterpret_cast<uint4*>(p.seg_copy + x * p.ld_copy + d.cbase + c0);
+              cp[0] = w[0];
+              cp[1] = w[1];
+            }
           }
         } else {
           const long long col = d.cbase + row_in_tile;
@@ -1078,7 +1148,7 @@ static bool map_mn(CUtensorMap* m, const aal_mat& t, int qv, int aw, int extent,
 // Output map for the TMA-store epilogue: 32 rows x 16 columns per store
 // (32-byte swizzle), or 16 rows x 32 columns when TMEM lanes are columns.
 static bool out_map(Params& p, const aal_mat& out, int qv) {
-  p.tma_store = (p.accumulate || p.swiglu_bwd) ? 0 : 1;
+  p.tma_store = (p.accumulate || p.swiglu_bwd || p.seg_mode) ? 0 : 1;
   if (!p.tma_store) return true;
   if (p.swap) return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 32, 16, 0);
   return make_map(&p.mapOut, out.ptr, out.rows, out.cols, out.ld, qv, 16, 32, 32);
@@ -1248,15 +1318,25 @@ static void schedule_tiles(Params& p, int grid) {
   p.use_order = 1;
 }
 
+// AAL_TEST_STALL=1 in the environment turns on Params::test_stall for the
+// tcgen05 launches made while it is set (a test hook for the timeout path;
+// read at every launch so that a test can switch it off again).
+static int test_stall_enabled() {
+  const char* e = getenv("AAL_TEST_STALL");
+  return (e && e[0] == '1') ? 1 : 0;
+}
+
 template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false>
 static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (ntiles <= 0) return AAL_OK;
   if (ntiles > INT_MAX) return AAL_ERR_UNSUPPORTED;
   p.ntiles = (int)ntiles;
-  order_pairs(p);
+  p.test_stall = test_stall_enabled();
+  if (!p.seg_mode) order_pairs(p);
   p.div_n1 = make_fastdiv((uint32_t)p.n1);
   p.div_n3 = make_fastdiv((uint32_t)p.n3);
   p.div_qm1 = make_fastdiv((uint32_t)(p.q > 1 ? p.q - 1 : 1));
+  p.div_qn3 = make_fastdiv((uint32_t)(p.q * p.n3));
   const size_t smem = (size_t)p.stages * p.stage_bytes + kEpiSmem + 1024;
   static unsigned long long attr_set = 0;  // one bit per device ordinal
   int dev = 0;
@@ -1272,7 +1352,8 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   const int sms = num_sms();
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    schedule_tiles(p, grid);
+    if (!p.seg_mode) schedule_tiles(p, grid);
+    else p.use_order = 0;
     k_tc<A_MN, B_MN, DUAL, false><<<grid, kThreads, smem, s>>>(p);
     note_launch();
     return cuda_status(cudaGetLastError());
@@ -1433,6 +1514,71 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
   p.n3 = (int)(bo / 128);
   ntiles = (long long)q * p.n2 * p.n3;
   return dual ? launch<true, false, 2>(p, ntiles, s) : launch<true, false, 0>(p, ntiles, s);
+}
+
+// Segment mode of the forward ops: Xg holds the rows gathered type by type
+// (tile table, count and permutation on the device), so a type's rows are
+// contiguous whatever the positions or explicit types were; Y receives row
+// perm[x] for gathered row x, and ``copy`` (if given) the same tiles in the
+// gathered order.  ``tmax`` bounds the table length.
+aal_status tc_project_seg(int law, int q, long long rows, const aal_mat& Xg, const aal_mat& Wg,
+                          const aal_mat* Wu, const aal_mat& Y, const int4* tiles, const int* count,
+                          const int* perm, int tmax, const aal_mat* copy, cudaStream_t s) {
+  if (!is_sm100()) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(Xg) || !tc_aligned(Wg) || !tc_aligned(Y) || (Wu && !tc_aligned(*Wu)) ||
+      (copy && !tc_aligned(*copy)))
+    return AAL_ERR_UNSUPPORTED;
+  const long long bi = Xg.cols / q, bo = Wg.cols / q;
+  if (bi % 16 || bo % 16 || bi > INT_MAX || bo > INT_MAX || rows > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  const bool dual = Wu != nullptr;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.law = law;
+  p.q = q;
+  p.qv = 1;
+  p.Mq = rows;
+  p.Mall = rows;
+  p.op = dual ? OP_SWIGLU : OP_FWD;
+  p.bi = (int)bi;
+  p.bo = (int)bo;
+  p.swiglu = dual;
+  p.out = (__nv_bfloat16*)Y.ptr;
+  p.ldo = Y.ld;
+  p.seg_mode = 1;
+  p.seg_tiles = tiles;
+  p.seg_count = count;
+  p.seg_perm = perm;
+  if (copy) {
+    p.seg_copy = (__nv_bfloat16*)copy->ptr;
+    p.ld_copy = copy->ld;
+  }
+  const int n = pick_n(bo, dual ? 128 : 256);
+  if (!n) return AAL_ERR_UNSUPPORTED;
+  p.swap = 0;
+  p.xr = 128;
+  p.wn = n;
+  p.n_mma = n;
+  p.a_rows = 128;
+  p.b_rows = n;
+  p.b_aw = n % 64 == 0 ? 64 : 16;
+  p.idesc = make_idesc(128, n, false, true);
+  p.fuse_b = dual && p.b_aw == 64 && 2 * n <= 256;
+  p.idesc2 = p.fuse_b ? make_idesc(128, 2 * n, false, true) : 0;
+  if (!finish_plan(p, dual ? 1 : 0)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapA[0], Xg, 1, 128)) return AAL_ERR_UNSUPPORTED;
+  int mg1 = 1;
+  if (!map_mn(&p.mapB[0], Wg, 1, p.b_aw, p.b_rows, &p.b_merged)) return AAL_ERR_UNSUPPORTED;
+  if (dual && !map_mn(&p.mapB[1], *Wu, 1, p.b_aw, p.b_rows, &mg1)) return AAL_ERR_UNSUPPORTED;
+  if (!mg1 && p.b_merged) {
+    p.b_merged = 0;
+    if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+  }
+  if (!out_map(p, Y, 1)) return AAL_ERR_UNSUPPORTED;
+  p.n1 = 1;
+  p.n2 = q;
+  p.n3 = (int)(bo / n);
+  const long long ntiles = (long long)tmax * q * p.n3;
+  return dual ? launch<false, true, 1>(p, ntiles, s) : launch<false, true, 0>(p, ntiles, s);
 }
 
 aal_status tc_project(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,

@@ -1021,6 +1021,8 @@ def measure(name, args, dist_on, world, rank, peaks):
     status = aal.aal_get_device_status()
     if status != aal.AAL_OK:
         raise SystemExit(f"{name}: device status after the timed region: {aal.status_string(status)}")
+    # read now: the graphs' event pairs hold the timed region's last replay of
+    # each graph until the hot leg below replays them again
     live = [e[1].elapsed_time(e[2]) for ev in evs for e in ev if e is not None]
     total_ms = _max_over_ranks(total_ms, dist_on)
     value, ms = job_throughput(total_ms, args.steps, world, wl.exec_flops)

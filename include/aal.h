@@ -190,9 +190,23 @@ AAL_API aal_status aal_decode_matvec(int32_t law, int32_t q, const int64_t* posi
  *   positions: device int64 [B]; x [B, D]; Wg, Wu [D, F]; Wd [F, D];
  *   h [B, F] (caller's workspace, overwritten with the activation, bf16 or
  *   fp32 like the inputs); y [B, D] (overwritten).
- * Two launches: gate, up and the activation in one kernel, then the down
- * decode.  An entry with a negative position is skipped (its rows of h and
- * y are not written) and the device status reports AAL_ERR_DEVICE_BOUNDS.
+ * Two launches: gate, up and the activation in one tensor-core decode
+ * kernel (one launch per 128 entries), then the down decode; up to 16
+ * entries the down decode is a programmatic dependent launch that fetches
+ * its weights while the first kernel runs and waits for h on the device.
+ * With AAL_FFN_DECODE_FUSED=1 in the environment the step is instead one
+ * launch per 128 entries where the shape allows it (bf16, q <= 64, D / q and
+ * F / q multiples of 16, 16-byte aligned rows, D / 16 below the SM count):
+ * CTAs owning 16 columns of h run gate, up and the activation; CTAs owning 16
+ * columns of y stage their columns of Wd meanwhile, wait in a grid barrier
+ * (bounded; a wait that runs out records AAL_ERR_DEVICE_TIMEOUT) and finish
+ * the down projection.  That barrier uses one of 64 slots of the library's
+ * device memory, taken round robin per launch: at most 64 such launches may
+ * run concurrently on one device (a launch captured into a CUDA graph keeps
+ * its slot).  It is opt-in because on B200 it measured slower than the two
+ * launches (12.9 against 8.4 us per step at one entry).
+ * An entry with a negative position is skipped (its rows of h and y are not
+ * written) and the device status reports AAL_ERR_DEVICE_BOUNDS.
  * Errors: AAL_ERR_INVALID_ARG for inconsistent shapes or a missing
  * positions array, AAL_ERR_UNSUPPORTED for mixed dtypes.
  */
@@ -238,6 +252,41 @@ AAL_API aal_status aal_swiglu_decode_noalloc(int32_t law, int32_t q, const int64
  */
 AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat W,
                               aal_mat Z, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Workspace for explicit and ragged row types                             */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * The tensor-core path reads the rows of one type through a strided view,
+ * which needs position-derived types with seq_len and the row count both
+ * multiples of q.  For explicit types, or sequences that do not line up
+ * (agihunt.info digest, Transformer-mapping paragraph: the type follows the
+ * absolute position, so any packing is legal), aal_project_fwd and
+ * aal_swiglu_fwd first sort the rows by type on the device into a caller
+ * workspace and then run the tensor-core path on the sorted rows, writing
+ * every output row back to its place.  Without a large enough workspace
+ * those calls take the general CUDA path (AAL_PATH_TENSOR: they fail with
+ * AAL_ERR_UNSUPPORTED).  The backward calls always take the general path for
+ * such rules.
+ *
+ * aal_workspace_size: bytes the call needs for ``rows`` rows; call is
+ * AAL_CALL_PROJECT_FWD (d_in = din, d_hidden unused) or AAL_CALL_SWIGLU_FWD
+ * (d_in = D, d_hidden = F).  0 when the rule needs none, -1 for invalid
+ * arguments.  Roughly rows * (d_in [+ d_hidden]) * 2 + rows * 4 bytes.
+ *
+ * aal_set_workspace: device memory the following calls of this host thread
+ * may use (NULL or 0 bytes: none).  The pointer must be 256-byte aligned
+ * (AAL_ERR_ALIGNMENT otherwise); the library does not own it, and the
+ * caller keeps it alive and unused by other work until the calls using it
+ * have completed on their streams.  Calls that overlap on the GPU must not
+ * share a workspace.  Supported: bf16, q <= 256, 16-byte aligned rows,
+ * din / q and dout / q multiples of 16.
+ */
+enum { AAL_CALL_PROJECT_FWD = 1, AAL_CALL_SWIGLU_FWD = 2 };
+AAL_API int64_t aal_workspace_size(int32_t call, int32_t law, int32_t q, aal_row_type_rule rule,
+                           int64_t rows, int64_t d_in, int64_t d_hidden);
+AAL_API aal_status aal_set_workspace(void* device_ptr, uint64_t bytes);
 
 /* ---------------------------------------------------------------------- */
 /* Host-side table queries (integer, no GPU needed)                        */
@@ -304,11 +353,13 @@ AAL_API int32_t aal_last_path(void);
  * aal_swiglu_decode), AAL_KERNEL_DECODE_GATE_UP (7, the gate/up/SiLU decode
  * kernel of aal_swiglu_decode), AAL_KERNEL_SWIGLU_BWD (8, the dH kernel of
  * aal_swiglu_bwd with the SiLU' chain; aal_swiglu_bwd's other launches use
- * the PROJECT, BWD_DX and BWD_DW kinds).
+ * the PROJECT, BWD_DX and BWD_DW kinds), AAL_KERNEL_FFN_DECODE (9, the
+ * one-launch FFN decode kernel of aal_swiglu_decode; with more than 128
+ * entries the pair brackets all of the call's launches).
  */
 enum { AAL_KERNEL_PROJECT = 1, AAL_KERNEL_GATE_UP = 2, AAL_KERNEL_BWD_DX = 3,
        AAL_KERNEL_BWD_DW = 4, AAL_KERNEL_SQUARE = 5, AAL_KERNEL_DECODE = 6,
-       AAL_KERNEL_DECODE_GATE_UP = 7, AAL_KERNEL_SWIGLU_BWD = 8 };
+       AAL_KERNEL_DECODE_GATE_UP = 7, AAL_KERNEL_SWIGLU_BWD = 8, AAL_KERNEL_FFN_DECODE = 9 };
 AAL_API aal_status aal_set_timing_events(int32_t kernel, void* before, void* after);
 
 /* Number of kernels launched by compute calls on this thread since the last

@@ -27,8 +27,24 @@ def packed_types(law, q, M, seq_len, offset=0):
     return oracle.row_types(law, q, inputs.packed_positions(M, seq_len, offset))
 
 
+class workspace:
+    """Context manager: a device workspace of the size the call needs, set for
+    this thread (aal_set_workspace) while the block runs."""
+
+    def __init__(self, call, law, q, rule, rows, d_in, d_hidden=0, extra=0):
+        self.n = aal.aal_workspace_size(call, law, q, rule, rows, d_in, d_hidden) + extra
+
+    def __enter__(self):
+        self.buf = torch.empty(max(self.n, 256), dtype=torch.uint8, device="cuda")
+        aal.aal_set_workspace(self.buf)
+        return self
+
+    def __exit__(self, *a):
+        aal.aal_set_workspace(None)
+
+
 def run_project(law, q, M, din, dout, dtype, seq_len=None, offset=0, explicit=False, seed=0,
-                policy=aal.AAL_PATH_AUTO):
+                policy=aal.AAL_PATH_AUTO, ws=False):
     ins = inputs.projection_inputs(M, din, dout, seed=seed, dtype=dtype)
     X, W = dev(ins["X"]), dev(ins["W"])
     Y = torch.full((M, dout), float("nan"), dtype=X.dtype, device="cuda")
@@ -43,8 +59,13 @@ def run_project(law, q, M, din, dout, dtype, seq_len=None, offset=0, explicit=Fa
         types = packed_types(law, q, M, seq_len, offset)
     aal.aal_set_path_policy(policy)
     try:
-        aal.aal_project_fwd(law, q, rule, X, W, Y)
-        torch.cuda.synchronize()
+        if ws:
+            with workspace(aal.AAL_CALL_PROJECT_FWD, law, q, rule, M, din):
+                aal.aal_project_fwd(law, q, rule, X, W, Y)
+                torch.cuda.synchronize()
+        else:
+            aal.aal_project_fwd(law, q, rule, X, W, Y)
+            torch.cuda.synchronize()
         path = aal.aal_last_path()
     finally:
         aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
@@ -78,20 +99,30 @@ def run_square(law, q, n, dtype, seed=0, policy=aal.AAL_PATH_AUTO):
 
 
 def run_swiglu(law, q, M, D, F, dtype, seq_len, w_sigma_rule="din", seed=0,
-               policy=aal.AAL_PATH_AUTO, rows=None):
+               policy=aal.AAL_PATH_AUTO, rows=None, ws=False, explicit=False):
     ins = inputs.swiglu_inputs(D, F, M, seed=seed, dtype=dtype, w_sigma_rule=w_sigma_rule)
     X, Wg, Wu, Wd = (dev(ins[k]) for k in ("X", "Wg", "Wu", "Wd"))
     H = torch.full((M, F), float("nan"), dtype=X.dtype, device="cuda")
     Y = torch.full((M, D), float("nan"), dtype=X.dtype, device="cuda")
-    rule = aal.row_rule(seq_len=seq_len)
+    if explicit:
+        tv = inputs.Stream(seed + 1).labels(M, q)
+        rule = aal.row_rule(types=torch.from_numpy(tv).cuda())
+        types = tv.astype(np.int64)
+    else:
+        rule = aal.row_rule(seq_len=seq_len)
+        types = packed_types(law, q, M, seq_len)
     aal.aal_set_path_policy(policy)
     try:
-        aal.aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y)
-        torch.cuda.synchronize()
+        if ws:
+            with workspace(aal.AAL_CALL_SWIGLU_FWD, law, q, rule, M, D, F):
+                aal.aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y)
+                torch.cuda.synchronize()
+        else:
+            aal.aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y)
+            torch.cuda.synchronize()
         path = aal.aal_last_path()
     finally:
         aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
-    types = packed_types(law, q, M, seq_len)
     if rows is None:
         Href, Yref = oracle.swiglu(law, q, types, ins["X"].f64, ins["Wg"].f64, ins["Wu"].f64, ins["Wd"].f64)
         Hg, Yg = host64(H), host64(Y)

@@ -243,3 +243,24 @@ def test_binding_refuses_host_short_or_strided_index_tensors():
             aal.aal_project_fwd("Q", 2, rule, X, W, Y)
         with pytest.raises(ValueError, match=msg):
             aal.aal_project_bwd("Q", 2, rule, X, W, Y, X, W)
+
+
+def test_every_compute_binding_runs_an_empty_call(lib):
+    # all-empty tensors reach the library without a GPU (nothing is
+    # launched), so each Python wrapper's argument marshalling and status
+    # check run end to end here
+    import torch
+    z = torch.empty(0, 0, dtype=torch.bfloat16)
+    pos = torch.empty(0, dtype=torch.int64)
+    rule = aal.row_rule(seq_len=16)
+    aal.aal_project_fwd("Q", 2, rule, z, z, z)
+    aal.aal_swiglu_fwd("Q", 2, rule, z, z, z, z, z, z)
+    aal.aal_project_bwd("Q", 2, rule, z, z, z, z, None)
+    aal.aal_swiglu_bwd("Q", 2, rule, *([z] * 14))
+    aal.aal_decode_matvec("Q", 2, pos, z, z, z)
+    aal.aal_swiglu_decode("Q", 2, pos, z, z, z, z, z, z)
+    aal.aal_swiglu_decode_noalloc("Q", 2, pos, z, z, z, z, z)
+    aal.aal_square_product("Q", 2, z, z, z)
+    assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_FWD, "Q", 2, rule, 0, 8) == 0
+    assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_FWD, "Q", 2, aal.row_rule(seq_len=7), 10, 64) > 10 * 64 * 2
+    aal.aal_set_workspace(None)

@@ -155,6 +155,55 @@ def test_swiglu_decode_other_shapes(law, q, B, D, F, dtype, path):
     assert got == path
 
 
+@pytest.mark.parametrize("B,launches", [(1, 2), (64, 2), (128, 2), (200, 3)])
+def test_swiglu_decode_launches(B, launches):
+    # gate/up/SiLU decode (one launch per 128 entries), then the down decode
+    # chained to it by a programmatic dependent launch
+    s = inputs.Stream(330 + B)
+    D, F = 768, 1536
+    x = s.normal(B, D, 1.0, "bf16", want_f64=False).t.cuda()
+    Wg, Wu = (s.normal(D, F, D ** -0.5, "bf16", want_f64=False).t.cuda() for _ in range(2))
+    Wd = s.normal(F, D, F ** -0.5, "bf16", want_f64=False).t.cuda()
+    pos = torch.from_numpy(s.positions(B, 1536)).cuda()
+    h = torch.empty(B, F, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(B, D, dtype=torch.bfloat16, device="cuda")
+    aal.aal_launch_count(reset=True)
+    aal.aal_swiglu_decode("Q2xQ2", 4, pos, x, Wg, Wu, Wd, h, y)
+    assert aal.aal_launch_count(reset=True) == launches
+    assert aal.aal_get_device_status() == aal.AAL_OK
+
+
+_ONE_LAUNCH_CHILD = r"""
+import sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
+from gpu_cases import TOL, run_swiglu_decode
+import associative_algebra_block_b200 as aal
+for B, launches in ((1, 1), (8, 1), (64, 1), (128, 1), (200, 2)):
+    aal.aal_launch_count(reset=True)
+    eh, ey, path = run_swiglu_decode('Q2xQ2', 4, B, 768, 1536, 'bf16', seed=340 + B)
+    assert path == aal.AAL_PATH_DECODE and eh <= TOL['bf16'] and ey <= TOL['bf16'], (B, eh, ey, path)
+    assert aal.aal_launch_count(reset=True) == launches, B
+for t in (0, 3):
+    eh, ey, _ = run_swiglu_decode('Q2xQ2', 4, 1, 768, 1536, 'bf16', seed=360 + t, same_type=t)
+    assert eh <= TOL['bf16'] and ey <= TOL['bf16'], (t, eh, ey)
+eh, ey, _ = run_swiglu_decode('Q', 16, 33, 2048, 1024, 'bf16', seed=370)
+assert eh <= TOL['bf16'] and ey <= TOL['bf16'], (eh, ey)
+print('ok')
+"""
+
+
+def test_one_launch_ffn_decode_parity():
+    # the opt-in one-launch FFN decode (gate/up CTAs and down CTAs in one
+    # grid, meeting in a bounded grid barrier)
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _ONE_LAUNCH_CHILD, root], capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, AAL_FFN_DECODE_FUSED="1"))
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
 def test_swiglu_decode_negative_position():
     s = inputs.Stream(7)
     x = s.normal(3, 128, 1.0, "bf16")
@@ -390,3 +439,100 @@ def test_cta_pair_mode_parity():
     r = subprocess.run([sys.executable, "-c", _PAIR_CHILD, root], capture_output=True, text=True,
                        timeout=600, env=dict(os.environ, AAL_TC_PAIR="1"))
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
+# ------------------------------------------------- bounded waits run out
+_STALL_CHILD = r"""
+import os, sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
+import torch
+from gpu_cases import TOL, run_project
+import associative_algebra_block_b200 as aal
+from associative_algebra_block_b200 import inputs
+X = inputs.projection_inputs(512, 512, 512, seed=3)["X"].t.cuda()
+W = inputs.projection_inputs(512, 512, 512, seed=4)["W"].t.cuda()
+Y = torch.zeros(512, 512, dtype=torch.bfloat16, device="cuda")
+os.environ["AAL_TEST_STALL"] = "1"
+aal.aal_set_path_policy(aal.AAL_PATH_TENSOR)
+aal.aal_project_fwd("Q", 4, aal.row_rule(seq_len=512), X, W, Y)
+st = aal.aal_get_device_status()
+del os.environ["AAL_TEST_STALL"]
+aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
+assert st == aal.AAL_ERR_DEVICE_TIMEOUT, st
+assert aal.aal_get_device_status() == aal.AAL_OK  # cleared by the read
+# the context is still usable: the same kernel, unstalled, matches the oracle
+err, path = run_project("Q", 4, 512, 512, 512, "bf16", seq_len=512, policy=aal.AAL_PATH_TENSOR)
+assert path == aal.AAL_PATH_TENSOR and err <= TOL["bf16"], (err, path)
+print("ok")
+"""
+
+
+def test_tcgen05_wait_that_runs_out_reports_timeout_and_returns():
+    # The test hook makes the MMA thread wait on a barrier nothing arrives on,
+    # bounded at 50 ms: the kernel records AAL_ERR_DEVICE_TIMEOUT, lets its
+    # copies land, frees TMEM and returns; the next call works normally.
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k != "AAL_TEST_STALL"}
+    r = subprocess.run([sys.executable, "-c", _STALL_CHILD, root], capture_output=True, text=True,
+                       timeout=600, env=env)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
+# ------------------------------------- explicit and ragged row types, tensor path
+# With a workspace set, explicit types and sequences that are not whole
+# multiples of q run on the tensor cores: rows sorted by type on the device,
+# the tcgen05 kernel in segment mode, outputs written back to their rows.
+@pytest.mark.parametrize("law,q,M,din,dout,seq_len,explicit", [
+    ("Q", 16, 2048, 2048, 768, None, True),        # expert shape, explicit types
+    ("Q", 16, 2048, 768, 2048, None, True),
+    ("Q2xQ2", 4, 12288, 768, 1536, None, True),    # pilot shape, explicit types
+    ("Q2xQ2", 4, 12288, 768, 1536, 1537, False),   # sequences of 1537 positions
+    ("Q", 8, 1003, 256, 512, 37, False),           # ragged rows and sequences
+    ("Q", 32, 333, 4096, 2048, None, True),        # few rows per type (partial tiles)
+    ("Q", 4, 7, 128, 256, None, True),             # fewer rows than types
+])
+def test_explicit_and_ragged_types_tensor_path(law, q, M, din, dout, seq_len, explicit):
+    err, path = run_project(law, q, M, din, dout, "bf16", seq_len=seq_len, explicit=explicit,
+                            seed=M + q, ws=True, policy=TENSOR)
+    assert err <= TOL["bf16"] and path == TENSOR, (err, path)
+
+
+@pytest.mark.parametrize("law,q,M,D,F,explicit,seq_len", [
+    ("Q2xQ2", 4, 3000, 768, 1536, True, None),
+    ("Q", 16, 2048, 2048, 768, False, 2047),
+])
+def test_explicit_and_ragged_types_swiglu_tensor_path(law, q, M, D, F, explicit, seq_len):
+    eh, ey, path = run_swiglu(law, q, M, D, F, "bf16", seq_len=seq_len or M, seed=q + M, ws=True,
+                              explicit=explicit, policy=TENSOR)
+    assert eh <= TOL["bf16"] and ey <= TOL["bf16"] and path == TENSOR, (eh, ey, path)
+
+
+def test_explicit_types_without_workspace_take_the_general_path():
+    err, path = run_project("Q", 8, 333, 128, 256, "bf16", explicit=True)
+    assert err <= TOL["bf16"] and path == aal.AAL_PATH_GENERAL
+    with pytest.raises(aal.AalError):
+        run_project("Q", 8, 333, 128, 256, "bf16", explicit=True, policy=TENSOR)
+
+
+def test_segment_path_skips_rows_with_an_invalid_type():
+    from gpu_cases import workspace
+    q, M, din, dout = 4, 300, 128, 256
+    X = torch.randn(M, din, device="cuda").to(torch.bfloat16)
+    W = torch.randn(din, dout, device="cuda").to(torch.bfloat16)
+    Y = torch.zeros(M, dout, dtype=torch.bfloat16, device="cuda")
+    types = torch.randint(0, q, (M,), dtype=torch.int32, device="cuda")
+    types[17] = -3
+    rule = aal.row_rule(types=types)
+    with workspace(aal.AAL_CALL_PROJECT_FWD, "Q", q, rule, M, din):
+        aal.aal_project_fwd("Q", q, rule, X, W, Y)
+        torch.cuda.synchronize()
+    assert aal.aal_last_path() == TENSOR
+    assert aal.aal_get_device_status() == aal.AAL_ERR_DEVICE_BOUNDS
+    assert torch.all(Y[17] == 0)
+    keep = torch.arange(M, device="cuda") != 17
+    tv = types.cpu().numpy().astype(np.int64)
+    ref = oracle.project("Q", q, tv[keep.cpu().numpy()], host64(X)[keep.cpu().numpy()], host64(W))
+    assert oracle.rel_err(host64(Y[keep]), ref) <= TOL["bf16"]
