@@ -50,7 +50,7 @@ from associative_algebra_block_b200 import inputs  # noqa: E402
 L2_BYTES = 126 * 2 ** 20
 METRIC = "executed BF16 TFLOP/s and % tensor peak per projection; speedup vs dense matmul"
 HEADLINE = "c5"
-ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c5")
+ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c4-explicit", "c2-explicit", "c5")
 
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture (the
 # summaries under profiles/ give the commands).  A figure is used only while
@@ -594,6 +594,103 @@ class SwigluFwdBwd:
             f"oracle SwiGLU forward + backward on {rows} of {self.M} rows (evenly strided, all row types)")
 
 
+class ExplicitTypes:
+    """A forward workload of the strided kind run with explicit row types
+    (uniform random per token) through the workspace path: rows sorted by
+    type on the device, the tensor cores in segment mode, outputs written
+    back in place.  ``swiglu``: the SwiGLU forward, else the two projections
+    D -> F and F -> D."""
+
+    has_e2e = False
+
+    def __init__(self, name, law, q, M, D, F, swiglu):
+        self.name, self.law, self.q, self.M, self.D, self.F, self.swiglu = name, law, q, M, D, F, swiglu
+        f1 = _exec_flops_proj(law, q, M, D, F)
+        f2 = _exec_flops_proj(law, q, M, F, D)
+        self.exec_flops = (2 * f1 + f2) if swiglu else (f1 + f2)
+        self.dense_flops = 2 * M * D * F * (3 if swiglu else 2)
+
+    def config(self):
+        what = "SwiGLU FFN fwd" if self.swiglu else f"projections {self.D}->{self.F} and {self.F}->{self.D}"
+        return {"workload": f"{self.name}: {self.law} q={self.q} {what}, M={self.M}, explicit random row "
+                            f"types (rows sorted by type into a workspace, tensor cores in segment mode)",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F}
+
+    def bytes_per_set(self):
+        e = 2
+        return e * (3 * self.D * self.F + self.M * (2 * self.D + 2 * self.F)) * 2
+
+    def setup(self, nsets, seed):
+        M, D, F = self.M, self.D, self.F
+        ins = inputs.swiglu_inputs(D, F, M, seed=seed, dtype="bf16", want_f64=False)
+        types = torch.from_numpy(inputs.Stream(seed + 9).labels(M, self.q)).cuda()
+        self.rule = aal.row_rule(types=types)
+        call = aal.AAL_CALL_SWIGLU_FWD if self.swiglu else aal.AAL_CALL_PROJECT_FWD
+        n = aal.aal_workspace_size(call, self.law, self.q, self.rule, M, max(D, F), F)
+        self.sets = []
+        for _ in range(nsets):
+            s = {k: ins[k].t.cuda() for k in ("X", "Wg", "Wu", "Wd")}
+            s["H"] = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+            s["Y"] = torch.empty(M, D, dtype=torch.bfloat16, device="cuda")
+            s["ws"] = torch.empty(n, dtype=torch.uint8, device="cuda")
+            self.sets.append(s)
+
+    def kernel_model(self, name):
+        """The timed slot brackets one whole call (the sort and gather
+        launches and the tensor-core launches): its algorithmic bytes are the
+        call's operands and results."""
+        M, D, F, e = self.M, self.D, self.F, 2
+        if self.swiglu:
+            return (2 * _exec_flops_proj(self.law, self.q, M, D, F) + _exec_flops_proj(self.law, self.q, M, F, D),
+                    e * (2 * M * D + 3 * D * F + M * F) + 4 * M)
+        return _exec_flops_proj(self.law, self.q, M, D, F), e * (M * D + D * F + M * F) + 4 * M
+
+    def timing_slots(self):
+        if self.swiglu:
+            return [("swiglu fwd call (sort, gather, gate/up, down)", aal.AAL_KERNEL_GATE_UP)]
+        return [(f"project call {self.D}->{self.F} (sort, gather, projection)", aal.AAL_KERNEL_PROJECT)]
+
+    def group_names(self):
+        return []
+
+    def step(self, i, ev=None, gev=None):
+        s = self.sets[i % len(self.sets)]
+        mark = _marker(ev)
+        aal.aal_set_workspace(s["ws"])
+        mark(0)
+        if self.swiglu:
+            aal.aal_swiglu_fwd(self.law, self.q, self.rule, s["X"], s["Wg"], s["Wu"], s["Wd"], s["H"], s["Y"])
+        else:
+            aal.aal_project_fwd(self.law, self.q, self.rule, s["X"], s["Wg"], s["H"])
+            aal.aal_project_fwd(self.law, self.q, self.rule, s["H"], s["Wd"], s["Y"])
+        aal.aal_set_workspace(None)
+
+    def dense_step(self, i):
+        s = self.sets[i % len(self.sets)]
+        torch.matmul(s["X"], s["Wg"], out=s["H"])
+        if self.swiglu:
+            torch.matmul(s["X"], s["Wu"], out=s["H"])
+        torch.matmul(s["H"], s["Wd"], out=s["Y"])
+
+    def oracle_sample(self, rows):
+        import oracle
+        rows = min(rows, self.M)
+        sel = np.arange(rows) * (self.M // rows)
+        types = inputs.Stream(9).labels(self.M, self.q).astype(np.int64)[sel]
+        ins = inputs.swiglu_inputs(self.D, self.F, self.M, seed=0, dtype="bf16")
+        X = ins["X"].f64[sel]
+
+        def run():
+            if self.swiglu:
+                oracle.swiglu(self.law, self.q, types, X, ins["Wg"].f64, ins["Wu"].f64, ins["Wd"].f64)
+            else:
+                H = oracle.project(self.law, self.q, types, X, ins["Wg"].f64)
+                oracle.project(self.law, self.q, types, H, ins["Wd"].f64)
+
+        return (self.exec_flops * rows) // self.M, run, (
+            f"oracle on {rows} of {self.M} rows (evenly strided) with the explicit types")
+
+
 class Square:
     """Fixed-block square product X * W (not row-typed).  The end-to-end leg
     treats W as the resident parameter and X as the step's input."""
@@ -693,6 +790,9 @@ WORKLOADS = {
     "c4": lambda: ProjFwdBwd("Qwen3-30B-A3B-expert-shaped FFN", "Q", 16, 2048, 2048, 768, 2048),
     "c5": lambda: Square("fixed-block square", "Q", 256, 32768),
     "c4-swiglu": lambda: SwigluFwdBwd("Qwen3-30B-A3B-expert-shaped SwiGLU FFN", "Q", 16, 2048, 2048, 768, 2048),
+    "c4-explicit": lambda: ExplicitTypes("Qwen3-30B-A3B-expert-shaped projections", "Q", 16, 2048, 2048, 768,
+                                         swiglu=False),
+    "c2-explicit": lambda: ExplicitTypes("Q2xQ2 110M pilot FFN", "Q2xQ2", 4, 12288, 768, 1536, swiglu=True),
 }
 
 
