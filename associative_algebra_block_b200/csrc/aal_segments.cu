@@ -7,8 +7,9 @@
 // absolute position, so any packing of sequences is legal), the rows are
 // first sorted by type on the device into a caller workspace: a per-block
 // histogram, one scan that also writes the tcgen05 kernel's tile table (a
-// type's rows in tiles of 128), and a scatter that records the permutation
-// and copies each row of X into its type's contiguous segment.  The tcgen05
+// type's rows in tiles of 128), a scatter that records the permutation, and
+// a wide gather that copies each row of X into its type's contiguous
+// segment.  The tcgen05
 // kernel then runs in segment mode and its epilogue writes every output row
 // back to its original place.  No host synchronisation: the tile count stays
 // on the device and tiles past it are empty.
@@ -18,7 +19,7 @@ namespace aal {
 namespace seg {
 
 constexpr int kThreads = 256;
-constexpr int kRowsPerBlock = 1024;
+constexpr int kRowsPerBlock = 4096;
 constexpr int kMaxQ = 256;
 
 struct Layout {
@@ -103,31 +104,77 @@ __global__ void __launch_bounds__(kThreads) k_seg_scan(long long G, int q, int* 
   }
 }
 
-// 3. each row takes the next place of its type's segment: the permutation
-//    records it and the row of X is copied there (16-byte vectors, one warp
-//    per row)
+// 3. each row takes the next place of its type's segment; the permutation
+//    records it
 __global__ void __launch_bounds__(kThreads) k_seg_scatter(RowTypes rt, long long rows, int q, const int* blk,
-                                                          int* perm, const __nv_bfloat16* X, long long ldx,
-                                                          int cols, __nv_bfloat16* Xg, long long ldg) {
+                                                          int* perm) {
   __shared__ int cur[kMaxQ];
-  __shared__ int dst[kRowsPerBlock];
   for (int i = threadIdx.x; i < q; i += kThreads) cur[i] = blk[(long long)blockIdx.x * q + i];
   __syncthreads();
   const long long r0 = (long long)blockIdx.x * kRowsPerBlock;
   const int nr = (int)(rows - r0 < kRowsPerBlock ? rows - r0 : kRowsPerBlock);
   for (int i = threadIdx.x; i < nr; i += kThreads) {
     const int t = row_type(rt, r0 + i);
-    const int d = t >= 0 ? atomicAdd(&cur[t], 1) : -1;
-    dst[i] = d;
-    if (d >= 0) perm[d] = (int)(r0 + i);
+    if (t >= 0) perm[atomicAdd(&cur[t], 1)] = (int)(r0 + i);
+  }
+}
+
+// 1-3 in one block, for calls whose rows all fit one block of the histogram:
+// histogram, segment starts, tile table and permutation without leaving the
+// CTA (one launch instead of three).
+constexpr int kSmallThreads = 1024;
+__global__ void __launch_bounds__(kSmallThreads) k_seg_sort_small(RowTypes rt, long long rows, int q, int* counts,
+                                                                  int4* tiles, int* perm) {
+  __shared__ int c[kMaxQ];
+  __shared__ int seg[kMaxQ + 1];
+  __shared__ int tst[kMaxQ + 1];
+  for (int i = threadIdx.x; i < q; i += kSmallThreads) c[i] = 0;
+  __syncthreads();
+  for (long long r = threadIdx.x; r < rows; r += kSmallThreads) {
+    const int t = row_type(rt, r);
+    if (t >= 0) atomicAdd(&c[t], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    seg[0] = 0;
+    tst[0] = 0;
+    for (int t = 0; t < q; ++t) {
+      seg[t + 1] = seg[t] + c[t];
+      tst[t + 1] = tst[t] + (c[t] + 127) / 128;
+    }
+    counts[q] = tst[q];
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < q; t += kSmallThreads) {
+    counts[t] = c[t];
+    const int nt = (c[t] + 127) / 128;
+    for (int i = 0; i < nt; ++i) tiles[tst[t] + i] = make_int4(t, seg[t] + 128 * i, seg[t] + c[t], 0);
+    c[t] = seg[t];  // now the next free place of type t
+  }
+  __syncthreads();
+  for (long long r = threadIdx.x; r < rows; r += kSmallThreads) {
+    const int t = row_type(rt, r);
+    if (t >= 0) perm[atomicAdd(&c[t], 1)] = (int)r;
+  }
+}
+
+// 4. the gathered copy: row d of Xg is row perm[d] of X (one warp per row,
+//    16-byte vectors; rows past the sorted count are left alone)
+__global__ void __launch_bounds__(kThreads) k_seg_gather(const int* counts, int q, const int* perm,
+                                                         const __nv_bfloat16* X, long long ldx, int cols,
+                                                         __nv_bfloat16* Xg, long long ldg, long long rows) {
+  __shared__ int s_total;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int t = 0; t < q; ++t) n += counts[t];
+    s_total = n;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nv = cols >> 3;
-  for (int i = warp; i < nr; i += kThreads / 32) {
-    const int d = dst[i];
-    if (d < 0) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(X + (r0 + i) * ldx);
-    uint4* out = reinterpret_cast<uint4*>(Xg + (long long)d * ldg);
+  for (long long d = (long long)blockIdx.x * (kThreads / 32) + warp; d < rows && d < s_total;
+       d += (long long)gridDim.x * (kThreads / 32)) {
+    const uint4* src = reinterpret_cast<const uint4*>(X + (long long)perm[d] * ldx);
+    uint4* out = reinterpret_cast<uint4*>(Xg + d * ldg);
     for (int v = lane; v < nv; v += 32) out[v] = src[v];
   }
 }
@@ -157,11 +204,18 @@ static aal_status seg_prepare(int q, const RowTypes& rt, long long rows, const a
   int4* tiles = (int4*)(ws + L.tiles);
   int* perm = (int*)(ws + L.perm);
   __nv_bfloat16* Xg = (__nv_bfloat16*)(ws + L.xg);
-  k_seg_hist<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk);
-  k_seg_scan<<<1, seg::kThreads, 0, s>>>(L.G, q, blk, counts, tiles);
-  k_seg_scatter<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk, perm, (const __nv_bfloat16*)X.ptr,
-                                                   X.ld, (int)X.cols, Xg, X.cols);
-  note_launch(3);
+  if (L.G == 1) {
+    k_seg_sort_small<<<1, kSmallThreads, 0, s>>>(rt, rows, q, counts, tiles, perm);
+  } else {
+    k_seg_hist<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk);
+    k_seg_scan<<<1, seg::kThreads, 0, s>>>(L.G, q, blk, counts, tiles);
+    k_seg_scatter<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk, perm);
+  }
+  const long long gb = (rows + seg::kThreads / 32 - 1) / (seg::kThreads / 32);
+  k_seg_gather<<<(unsigned)(gb < 4096 ? gb : 4096), seg::kThreads, 0, s>>>(counts, q, perm,
+                                                                          (const __nv_bfloat16*)X.ptr, X.ld,
+                                                                          (int)X.cols, Xg, X.cols, rows);
+  note_launch(L.G == 1 ? 2 : 4);
   return cuda_status(cudaGetLastError());
 }
 

@@ -148,6 +148,18 @@ struct Params {
   // segment, 0}; tile index = (j * q + k) * n3 + i3.  Output row x of the
   // gathered order is row seg_perm[x] of the caller's output; with seg_copy
   // the tile is also written, in the gathered order, to seg_copy.
+  // Ragged mode (forward projection whose blocks are not multiples of 16,
+  // e.g. 20 x 100): a segment is one input group a of gbi features.  Its A
+  // box holds ka features from the 16-byte aligned start below a * gbi (the
+  // group sits at offset (a * gbi) mod 8); its B boxes come from W seen as
+  // [groups][gbi rows][cols], started at row -offset, so every K position
+  // outside the group reads as zero and the neighbours' features in A are
+  // multiplied by zeros.  A tile spans N columns from the 16-column aligned
+  // start below k * gbo; the epilogue writes the group's gbo columns only.
+  int ragged;
+  int gbi, gbo, ka;
+  uint32_t tx_bytes;   // bytes one stage's copies deliver
+  uint32_t b_lbo;      // MN-major B: bytes between 16-column atoms (ragged mode)
   int seg_mode;
   const int4* seg_tiles;
   const int* seg_count;
@@ -169,6 +181,7 @@ struct TileDesc {
   int rstride, roff;
   long long rlimit;
   long long cbase;
+  int vlo, vhi;    // tile columns the epilogue writes (ragged mode)
 };
 
 // ------------------------------------------------------------------ PTX glue
@@ -380,7 +393,7 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t addr, uint32_t lbo, uint3
   d |= (uint64_t)layout << 61;
   return d;
 }
-constexpr uint32_t kLayoutSW128 = 2, kLayoutSW32 = 6;
+constexpr uint32_t kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6;
 
 // Descriptor of an operand tile at shared address ``tile`` (K step 0) and the
 // amount a K step of 16 adds to it (the start-address field is in 16-byte
@@ -483,6 +496,8 @@ __device__ __forceinline__ void pair_of(const Params& p, int pr, int& p0, int& p
 
 // Segment mode: tile = (j * q + k) * n3 + i3 over the device tile table.
 __device__ __forceinline__ void describe_seg(const Params& p, int tile, TileDesc& d) {
+  d.vlo = 0;
+  d.vhi = INT_MAX;
   const int j = (int)fdiv((uint32_t)tile, p.div_qn3);
   const int rem = tile - j * p.q * p.n3;
   const int k = (int)fdiv((uint32_t)rem, p.div_n3);
@@ -523,6 +538,34 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
   d.rstride = 1;
   d.roff = 0;
   d.rlimit = LLONG_MAX;
+  d.vlo = 0;
+  d.vhi = INT_MAX;
+  if (p.ragged) {  // OP_FWD, not swapped: i0 class, i1 token block, i2 output group k
+    // law Q_q: S(t, t) = {t}, S(t, k) = {t, k}; a segment's k0 is the group
+    const int c = i0, k = i2, t = type_of_class(p, c);
+    d.seg[0].k0 = t < k ? t : k;
+    d.seg[1].k0 = t < k ? k : t;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      d.seg[j].len = p.ka;
+      d.seg[j].cls = c;
+      d.seg[j].map = 0;
+    }
+    d.nseg = t == k ? 1 : 2;
+    const int col0 = k * p.gbo, x0 = col0 & ~15;
+    d.a_f = i1 * p.xr;
+    d.a_c1 = 1;
+    d.b_f = x0;
+    d.b_c1 = 0;
+    d.rbase = d.a_f;
+    d.rstride = p.qv;
+    d.roff = c;
+    d.rlimit = p.Mq;
+    d.cbase = x0;
+    d.vlo = col0 - x0;
+    d.vhi = d.vlo + p.gbo;
+    return;
+  }
   switch (p.op) {
     case OP_FWD:
     case OP_SWIGLU: {  // i0 class, i1 token block, i2 output group k, i3 column block
@@ -699,8 +742,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const uint32_t base = smem0 + st * p.stage_bytes;
             const int kofs = sg.k0 + kc * 64;
             const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
-            if (lane == 0 && issuer) mbar_expect_tx(&full_bar[st], (PAIR ? 2u : 1u) * p.stage_bytes);
+            if (lane == 0 && issuer) mbar_expect_tx(&full_bar[st], (PAIR ? 2u : 1u) * p.tx_bytes);
             if (lane == 0) atomicMax(&s_last_chunk[st], (int)it);
+            if (!A_MN && B_MN && DUAL == 0 && !PAIR && p.ragged) {
+              // lane 0: the A box; lane 1: the B box (all atoms, ka rows from -oa)
+              const int a = sg.k0, oa = (a * p.gbi) & 7;
+              if (lane == 0)
+                tma_load(&p.mapA[0], base, &full_bar[st], a * p.gbi - oa, d.a_c1 ? sg.cls : 0, d.a_f);
+              else if (lane == 1)
+                tma_load4(&p.mapB[0], base + p.a_bytes, &full_bar[st], 0, -oa, a, d.b_f >> 4);
+            } else {
             const int na = DUAL == 2 ? 2 : 1;
             const int nb = (DUAL == 1 && !PAIR) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
@@ -745,6 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 }
               }
             }
+            }
           }
           __syncwarp();
           ++it;
@@ -779,9 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       const int na = DUAL == 2 ? 2 : 1;
       // Descriptors of stage 0 and their per-stage and per-K-step increments,
       // built once: the issue loop below only adds.
-      const uint64_t dA0 = operand_desc0<A_MN>(smem0, p.a_aw);
+      const bool rg = !A_MN && B_MN && DUAL == 0 && !PAIR && p.ragged;
+      const uint64_t dA0 = rg ? make_desc(smem0, 16, 16u * p.ka, p.ka == 32 ? kLayoutSW64 : kLayoutSW128)
+                              : operand_desc0<A_MN>(smem0, p.a_aw);
       const uint64_t dA1 = operand_desc0<A_MN>(smem0 + p.a_bytes, p.a_aw);
-      const uint64_t dB0 = operand_desc0<B_MN>(smem0 + na * p.a_bytes, p.b_aw);
+      const uint64_t dB0 = rg ? make_desc(smem0 + p.a_bytes, p.b_lbo, 8 * 32, kLayoutSW32)
+                              : operand_desc0<B_MN>(smem0 + na * p.a_bytes, p.b_aw);
       const uint64_t dB1 = operand_desc0<B_MN>(smem0 + na * p.a_bytes + p.b_bytes, p.b_aw);
       const uint64_t dstage = p.stage_bytes >> 4;
       const uint64_t kA = operand_kstep<A_MN>(p.a_aw), kB = operand_kstep<B_MN>(p.b_aw);
@@ -877,6 +932,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       if (!warp_wait(&tfull_bar[buf], use & 1u, &s_abort)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + buf * p.acc_cols;
+      // segment mode: the caller's row of this thread's TMEM lane, looked up
+      // once per tile (its load overlaps the first TMEM read)
+      int seg_row = 0;
+      if (p.seg_mode && !p.swap && d.rbase + row_in_tile < d.rlimit) seg_row = p.seg_perm[d.rbase + row_in_tile];
       const uint32_t tempty_addr =
           PAIR ? mapa_rank(smem_u32(&tempty_bar[buf]), 0) : smem_u32(&tempty_bar[buf]);
       const int nch = (p.n_mma / 16 + 1 - half) / 2;  // chunks c0 = half*16 + 32*i
@@ -908,7 +967,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             else mbar_arrive(&tempty_bar[buf]);
           }
         }
-        if (p.tma_store) {
+        if (p.tma_store && (c0 < d.vlo || c0 + 16 > d.vhi)) {
+          // ragged mode: a chunk at or past the edge of the group's columns;
+          // its columns inside the group go out as 8-byte stores (4 columns,
+          // when the edges fall on multiples of 4) or one by one
+          const long long x = d.rbase + row_in_tile;
+          if (!p.swap && x < d.rlimit && c0 + 16 > d.vlo && c0 < d.vhi) {
+            __nv_bfloat16* dst = p.out + (x * d.rstride + d.roff) * p.ldo + d.cbase + c0;
+            if (((d.vlo | d.vhi) & 3) == 0) {
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                if (c0 + 4 * g >= d.vlo && c0 + 4 * g + 4 <= d.vhi) {
+                  uint2 w;
+                  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&w);
+                  h[0] = __floats2bfloat162_rn(v[4 * g], v[4 * g + 1]);
+                  h[1] = __floats2bfloat162_rn(v[4 * g + 2], v[4 * g + 3]);
+                  *reinterpret_cast<uint2*>(dst + 4 * g) = w;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (c0 + j >= d.vlo && c0 + j < d.vhi) dst[j] = __float2bfloat16_rn(v[j]);
+            }
+          }
+        } else if (p.tma_store) {
           const uint32_t sb = stage_buf + (nstore & 1u) * 1024;
           if (nstore >= 2) {
             if (lane == 0) bulk_wait_read1();  // the buffer's previous store has read it
@@ -985,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             reinterpret_cast<uint4*>(p.out2 + off)[0] = w[0];
             reinterpret_cast<uint4*>(p.out2 + off)[1] = w[1];
           } else if (x < d.rlimit) {
-            const long long xo = p.seg_mode ? (long long)p.seg_perm[x] : x * d.rstride + d.roff;
+            const long long xo = p.seg_mode ? (long long)seg_row : x * d.rstride + d.roff;
             __nv_bfloat16* dst = p.out + xo * p.ldo + d.cbase + c0;
             if (p.accumulate) {
               uint4 o0 = reinterpret_cast<const uint4*>(dst)[0];
@@ -1145,6 +1228,23 @@ static bool map_mn(CUtensorMap* m, const aal_mat& t, int qv, int aw, int extent,
   return map_mnmajor(m, t, qv, aw);
 }
 
+// Ragged mode: W [din, dout] seen as [dout / 16 atoms][din / gbi groups]
+// [gbi rows][16 columns]; one box {16 columns, ka rows, 1 group, natoms}
+// lands in shared memory as the MN-major atoms the MMA reads (ka rows of 32
+// bytes each, 32-byte swizzle).  ka exceeds gbi: rows past the group, and
+// rows before it when the box starts at a negative row, read as zeros.
+static bool map_ragged_w(CUtensorMap* m, const aal_mat& w, int gbi, int ka, int natoms) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || w.rows % gbi || w.cols % 16) return false;
+  cuuint64_t dims[4] = {16u, (cuuint64_t)gbi, (cuuint64_t)(w.rows / gbi), (cuuint64_t)(w.cols / 16)};
+  cuuint64_t strides[3] = {(cuuint64_t)(w.ld * 2), (cuuint64_t)(w.ld * 2 * gbi), 32u};
+  cuuint32_t box[4] = {16u, (cuuint32_t)ka, 1u, (cuuint32_t)natoms};
+  cuuint32_t es[4] = {1u, 1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, w.ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output map for the TMA-store epilogue: 32 rows x 16 columns per store
 // (32-byte swizzle), or 16 rows x 32 columns when TMEM lanes are columns.
 static bool out_map(Params& p, const aal_mat& out, int qv) {
@@ -1202,6 +1302,17 @@ static bool finish_plan(Params& p, int dual, bool pair = false) {
   p.a_bytes = (uint32_t)p.a_rows * 128u;
   p.b_bytes = (uint32_t)p.b_rows * 128u;
   p.stage_bytes = na * p.a_bytes + nb * p.b_bytes;
+  if (p.ragged) {
+    // A: 128 rows of ka features; B: the atoms of 16 columns x ka rows.  The
+    // stride between stages stays a multiple of 1 KB (swizzle alignment).
+    p.a_bytes = 128u * (uint32_t)p.ka * 2u;
+    p.b_lbo = (uint32_t)p.ka * 32u;
+    p.b_bytes = (uint32_t)(p.n_mma / 16) * p.b_lbo;
+    p.tx_bytes = p.a_bytes + p.b_bytes;
+    p.stage_bytes = (p.tx_bytes + 1023u) & ~1023u;
+  } else {
+    p.tx_bytes = p.stage_bytes;
+  }
   p.stages = (kSmemBudget - kEpiSmem) / (int)p.stage_bytes;
   if (p.stages > kMaxStages) p.stages = kMaxStages;
   if (p.stages < 2) return false;
@@ -1415,8 +1526,48 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
   if (!tc_aligned(X) || !tc_aligned(Wg) || !tc_aligned(Y) || (Wu && !tc_aligned(*Wu)))
     return AAL_ERR_UNSUPPORTED;
   const long long bi = X.cols / q, bo = Wg.cols / q;
-  if (bi % 16 || bo % 16 || bi > INT_MAX || bo > INT_MAX) return AAL_ERR_UNSUPPORTED;
+  if (bi > INT_MAX || bo > INT_MAX) return AAL_ERR_UNSUPPORTED;
   const bool dual = Wu != nullptr;
+  if (bi % 16 || bo % 16) {
+    // Ragged mode (a forward projection with groups that are not multiples
+    // of 16): the A box spans ka >= offset + gbi features, the tile N >=
+    // column offset + gbo columns, over every group a and k.
+    if (dual || bi < 16 || law != AAL_LAW_Q) return AAL_ERR_UNSUPPORTED;
+    int oa = 0, oc = 0;
+    for (long long g = 0; g < q; ++g) {
+      oa = std::max(oa, (int)((g * bi) & 7));
+      oc = std::max(oc, (int)((g * bo) & 15));
+    }
+    const int ka = (int)((oa + bi + 15) / 16 * 16), n = (int)((oc + bo + 15) / 16 * 16);
+    if ((ka != 32 && ka != 64) || n > 256) return AAL_ERR_UNSUPPORTED;
+    Params p;
+    base_params(p, law, q, rt, rows);
+    p.op = OP_FWD;
+    p.ragged = 1;
+    p.gbi = (int)bi;
+    p.gbo = (int)bo;
+    p.ka = ka;
+    p.bi = (int)bi;
+    p.bo = (int)bo;
+    p.out = (__nv_bfloat16*)Y.ptr;
+    p.ldo = Y.ld;
+    p.swap = 0;
+    p.xr = 128;
+    p.wn = n;
+    p.n_mma = n;
+    p.a_rows = 128;
+    p.b_rows = n;
+    p.b_aw = 16;
+    p.idesc = make_idesc(128, n, false, true);
+    if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+    if (!make_map(&p.mapA[0], X.ptr, X.rows, X.cols, X.ld, q, ka, 128, ka * 2)) return AAL_ERR_UNSUPPORTED;
+    if (!map_ragged_w(&p.mapB[0], Wg, (int)bi, ka, n / 16)) return AAL_ERR_UNSUPPORTED;
+    if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = (int)((p.Mq + 127) / 128);
+    p.n2 = q;
+    p.n3 = 1;
+    return launch<false, true, 0>(p, (long long)q * p.n1 * p.n2, s);
+  }
   Params p;
   base_params(p, law, q, rt, rows);
   p.op = dual ? OP_SWIGLU : OP_FWD;

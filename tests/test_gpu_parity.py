@@ -536,3 +536,48 @@ def test_segment_path_skips_rows_with_an_invalid_type():
     tv = types.cpu().numpy().astype(np.int64)
     ref = oracle.project("Q", q, tv[keep.cpu().numpy()], host64(X)[keep.cpu().numpy()], host64(W))
     assert oracle.rel_err(host64(Y[keep]), ref) <= TOL["bf16"]
+
+
+# --------------------------------- ragged blocks (groups not multiples of 16)
+# The tensor-core path's ragged mode: an input group of 20 features is read
+# from the 16-byte aligned start below it with the weight rows outside the
+# group read as zeros; output tiles span the 16-column aligned window around
+# the group and only the group's columns are written.
+@pytest.mark.parametrize("q,M,din,dout,seq_len", [
+    (16, 2048, 320, 1600, 2048),    # 20 x 100 blocks, as in the Qwen3-32B shape
+    (16, 3200, 320, 1600, 3200),    # 200 tokens per type: partial token tiles
+    (8, 1024, 192, 320, 1024),      # 24 x 40 blocks
+    (4, 512, 80, 208, 512),         # 20 x 52 blocks
+])
+def test_ragged_blocks_tensor_path(q, M, din, dout, seq_len):
+    err, path = run_project("Q", q, M, din, dout, "bf16", seq_len=seq_len, seed=din + dout, policy=TENSOR)
+    assert err <= TOL["bf16"] and path == TENSOR, (err, path)
+
+
+def test_qwen3_32b_shaped_projection_sampled_rows():
+    # M = 32768, D = 5120 -> F = 25600, q = 256 (20 x 100 blocks): NaN-prefilled
+    # output; every row finite, and 64 rows (all of one token block, plus rows
+    # of other types) against the oracle over all 25600 columns
+    law, q, M, D, F = "Q", 256, 32768, 5120, 25600
+    ins = inputs.projection_inputs(M, D, F, seed=32, dtype="bf16", want_f64=False)
+    X, W = ins["X"].t.cuda(), ins["W"].t.cuda()
+    Y = torch.full((M, F), float("nan"), dtype=torch.bfloat16, device="cuda")
+    aal.aal_project_fwd(law, q, aal.row_rule(seq_len=M), X, W, Y)
+    torch.cuda.synchronize()
+    assert aal.aal_last_path() == TENSOR
+    assert aal.aal_get_device_status() == aal.AAL_OK
+    assert bool(torch.isfinite(Y).all())
+    rows = np.concatenate([np.arange(0, 256, 8), np.array([257, 1000, 4095, 9999, 16384, 20000, 30001,
+                                                           32767]), np.arange(32512, 32768, 11)])[:64]
+    types = oracle.row_types(law, q, inputs.packed_positions(M, M))
+    Wf = ins["W"].t.to(torch.float64).numpy()
+    Xs = ins["X"].t[torch.as_tensor(rows)].to(torch.float64).numpy()
+    ref = oracle.project(law, q, types[rows], Xs, Wf)
+    got = host64(Y[torch.as_tensor(rows, device="cuda")])
+    assert oracle.rel_err(got, ref) <= TOL["bf16"]
+
+
+def test_qwen3_1_7b_shaped_projection_full():
+    # M = 2048, D = 2048 -> F = 6144, q = 32 (64 x 192 blocks)
+    err, path = run_project("Q", 32, 2048, 2048, 6144, "bf16", seq_len=2048, seed=17)
+    assert err <= TOL["bf16"] and path == TENSOR, err
