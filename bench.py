@@ -59,14 +59,14 @@ ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c4-explicit", "c2-explicit", "qwe
 # null.
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
-    ("c2", "gate_up"): ("5c4e5cfd1c76a48e07f5320532c225e01a72d9b57aa9e792520f5fc1f1cf2123",
-                        23667968 + 749312, "aal_tc.cu"),
-    ("c2", "down"): ("5c4e5cfd1c76a48e07f5320532c225e01a72d9b57aa9e792520f5fc1f1cf2123",
-                     40178688 + 912896, "aal_tc.cu"),
-    ("c2", "decode gate_up B=64"): ("5666616e0a8887abcc355dc9a3026e1f8a01385ef66e4f33975abdff2957c51c",
-                                    4854272, "aal_decode.cu"),
-    ("c2", "decode down B=64"): ("5666616e0a8887abcc355dc9a3026e1f8a01385ef66e4f33975abdff2957c51c",
-                                 2587392, "aal_decode.cu"),
+    # c5: captured at n = 16384 (--config c5-n16384), x 4 for n = 32768 (4 x the tiles and bytes)
+    ("c5", "square product"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 4 * (1082815000 + 507556096), "aal_tc.cu"),
+    ("c5-n16384", "square product"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 1082815000 + 507556096, "aal_tc.cu"),
+    ("c2", "gate_up"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 23675136 + 1578240, "aal_tc.cu"),
+    ("c2", "down"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 40183808 + 1218816, "aal_tc.cu"),
+    ("c3", "gate_up"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 218600448 + 35601152, "aal_tc.cu"),
+    ("c2", "decode gate_up B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 4746240, "aal_decode.cu"),
+    ("c2", "decode down B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 2385152, "aal_decode.cu"),
 }
 
 
@@ -865,6 +865,9 @@ WORKLOADS = {
                                w_sigma_rule="D", decode_batches=()),
     "c4": lambda: ProjFwdBwd("Qwen3-30B-A3B-expert-shaped FFN", "Q", 16, 2048, 2048, 768, 2048),
     "c5": lambda: Square("fixed-block square", "Q", 256, 32768),
+    # the square-product kernel on a quarter of the c5 bytes (n = 16384, q = 128,
+    # the same b = 128): a case small enough for full ncu captures
+    "c5-n16384": lambda: Square("fixed-block square (profiling size)", "Q", 128, 16384),
     "c4-swiglu": lambda: SwigluFwdBwd("Qwen3-30B-A3B-expert-shaped SwiGLU FFN", "Q", 16, 2048, 2048, 768, 2048),
     "qwen3-1.7b": lambda: Projection("Qwen3-1.7B-shaped expanding projection", "Q", 32, 2048, 2048, 6144, 2048),
     "qwen3-32b": lambda: Projection("Qwen3-32B-shaped expanding projection", "Q", 256, 32768, 5120, 25600, 32768),
