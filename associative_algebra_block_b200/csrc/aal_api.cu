@@ -238,13 +238,13 @@ aal_status aal_swiglu_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_ma
                   });
     if (st != AAL_OK) return st;
     note();
-    // 3. dX = dG Wg^T + dU Wu^T over the table
-    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dG, Wg, dX, 0, s); },
-                  [&] { return simt_project_bwd_dx(law, q, rt, dG, Wg, dX, s); });
-    if (st != AAL_OK) return st;
-    note();
-    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dU, Wu, dX, 1, s); },
-                  [&] { return simt_project_bwd_dx(law, q, rt, dU, Wu, dX, s, 1); });
+    // 3. dX = dG Wg^T + dU Wu^T over the table: one tensor-core launch with
+    //    both products in the same accumulator, else two general passes
+    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_swiglu_bwd_dx(law, q, rt, M, dG, Wg, dU, Wu, dX, s); },
+                  [&] {
+                    aal_status e = simt_project_bwd_dx(law, q, rt, dG, Wg, dX, s);
+                    return e != AAL_OK ? e : simt_project_bwd_dx(law, q, rt, dU, Wu, dX, s, 1);
+                  });
     if (st != AAL_OK) return st;
     note();
   }

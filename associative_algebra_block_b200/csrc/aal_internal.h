@@ -113,6 +113,9 @@ aal_status tc_swiglu_gate_up(int law, int q, const RowTypes& rt, long long rows,
                              const aal_mat& Wg, const aal_mat& Wu, const aal_mat& H, cudaStream_t s);
 aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
                              const aal_mat& W, const aal_mat& dX, int accumulate, cudaStream_t s);
+aal_status tc_swiglu_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dG,
+                            const aal_mat& Wg, const aal_mat& dU, const aal_mat& Wu, const aal_mat& dX,
+                            cudaStream_t s);
 aal_status tc_swiglu_bwd_dh(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
                             const aal_mat& Wd, const aal_mat& G, const aal_mat& U,
                             const aal_mat& dG, const aal_mat& dU, cudaStream_t s);

@@ -648,7 +648,9 @@ __device__ __forceinline__ bool take_tile(const TileDesc* ring, uint64_t* full, 
 
 // --------------------------------------------------------------- the kernel
 // A_MN / B_MN: operand tiles stored MN-major (else K-major).
-// DUAL: 0 one MMA per K step; 1 two B operands (gate/up); 2 two A operands.
+// DUAL: 0 one MMA per K step; 1 two B operands (gate/up); 2 two A operands;
+// 3 two (A, B) pairs summed into one accumulator (the SwiGLU backward's
+// dX = dG Wg^T + dU Wu^T).
 // PAIR: the tile is computed by a CTA pair with tcgen05 cta_group::2 (M = 256);
 // each CTA loads its half of A's rows and of B's columns (for DUAL == 1, CTA r
 // loads B operand r), only the pair's first CTA issues MMAs and counts the
@@ -752,8 +754,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               else if (lane == 1)
                 tma_load4(&p.mapB[0], base + p.a_bytes, &full_bar[st], 0, -oa, a, d.b_f >> 4);
             } else {
-            const int na = DUAL == 2 ? 2 : 1;
-            const int nb = (DUAL == 1 && !PAIR) ? 2 : 1;
+            const int na = DUAL >= 2 ? 2 : 1;
+            const int nb = ((DUAL == 1 && !PAIR) || DUAL == 3) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
             const int nB = (B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1;  // boxes per B operand
             const int arow = PAIR ? (int)rank * 128 : 0;  // this CTA's half of the A tile
@@ -761,7 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             for (int bx = lane; bx < na * nA + nb * nB; bx += 32) {
               if (bx < na * nA) {
                 const int o = bx / nA, at = bx - o * nA;
-                const CUtensorMap* m = &p.mapA[DUAL == 2 ? o : sg.map];
+                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : sg.map];
                 const int c1 = d.a_c1 ? sg.cls : 0;
                 const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
                 if (A_MN && p.a_merged) {
@@ -779,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
                 // the MMA's B, or, with two B operands, all of operand r
                 const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
-                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : sg.map;
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : sg.map);
                 const CUtensorMap* m = &p.mapB[mop];
                 const int c1 = d.b_c1 ? sg.cls : 0;
                 const uint32_t dst =
@@ -828,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       // divisions, so the next MMAs follow the previous ones closely.
       uint32_t st = 0, ph = 0, tl = 0;
       bool ok = true;
-      const int na = DUAL == 2 ? 2 : 1;
+      const int na = DUAL >= 2 ? 2 : 1;
       // Descriptors of stage 0 and their per-stage and per-K-step increments,
       // built once: the issue loop below only adds.
       const bool rg = !A_MN && B_MN && DUAL == 0 && !PAIR && p.ragged;
@@ -879,6 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                   tc_mma(acc0, a0 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
                   if (DUAL == 1) tc_mma(acc1, a0 + ks * kA, b1 + ks * kB, p.idesc, accumulate);
                   if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
+                  if (DUAL == 3) tc_mma(acc0, a1 + ks * kA, b1 + ks * kB, p.idesc, 1u);
                 }
                 accumulate = 1;
               }
@@ -894,6 +897,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                   tc_mma(acc0, da, db, p.idesc, accumulate);
                   if (DUAL == 1) tc_mma(acc1, da, b1 + ks * kB, p.idesc, accumulate);
                   if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, db, p.idesc, accumulate);
+                  if (DUAL == 3) tc_mma(acc0, a1 + ks * kA, b1 + ks * kB, p.idesc, 1u);
                 }
                 accumulate = 1;
               }
@@ -1298,7 +1302,7 @@ static bool is_sm100() {
 
 // Fills the pipeline sizes and TMEM allocation; false if they do not fit.
 static bool finish_plan(Params& p, int dual, bool pair = false) {
-  const int na = dual == 2 ? 2 : 1, nb = (dual == 1 && !pair) ? 2 : 1;
+  const int na = dual >= 2 ? 2 : 1, nb = ((dual == 1 && !pair) || dual == 3) ? 2 : 1;
   p.a_bytes = (uint32_t)p.a_rows * 128u;
   p.b_bytes = (uint32_t)p.b_rows * 128u;
   p.stage_bytes = na * p.a_bytes + nb * p.b_bytes;
@@ -1316,7 +1320,7 @@ static bool finish_plan(Params& p, int dual, bool pair = false) {
   p.stages = (kSmemBudget - kEpiSmem) / (int)p.stage_bytes;
   if (p.stages > kMaxStages) p.stages = kMaxStages;
   if (p.stages < 2) return false;
-  p.acc_cols = p.n_mma * (dual ? 2 : 1);
+  p.acc_cols = p.n_mma * ((dual == 1 || dual == 2) ? 2 : 1);
   const int need = 2 * p.acc_cols;
   if (need > 512) return false;
   uint32_t cols = 32;
@@ -1786,6 +1790,42 @@ static aal_status bwd_dx_impl(int law, int q, const RowTypes& rt, long long rows
   p.n2 = q;
   p.n3 = (int)(bi / n);
   return launch<false, false, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+}
+
+// dX of the SwiGLU backward in one launch: dX = dG Wg^T + dU Wu^T through the
+// transposed table, both products of a tile accumulated in the same TMEM
+// accumulator (one rounding to bf16).
+aal_status tc_swiglu_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dG,
+                            const aal_mat& Wg, const aal_mat& dU, const aal_mat& Wu, const aal_mat& dX,
+                            cudaStream_t s) {
+  if (!is_sm100() || !position_rule_ok(rt, q, rows)) return AAL_ERR_UNSUPPORTED;
+  if (!tc_aligned(dG) || !tc_aligned(dU) || !tc_aligned(Wg) || !tc_aligned(Wu) || !tc_aligned(dX))
+    return AAL_ERR_UNSUPPORTED;
+  const long long bi = Wg.rows / q, bo = Wg.cols / q;
+  if (bi % 16 || bo % 16) return AAL_ERR_UNSUPPORTED;
+  Params p;
+  base_params(p, law, q, rt, rows);
+  p.op = OP_DX;
+  p.bi = (int)bi;
+  p.bo = (int)bo;
+  p.out = (__nv_bfloat16*)dX.ptr;
+  p.ldo = dX.ld;
+  const int n = pick_n(bi, 256);
+  if (!n) return AAL_ERR_UNSUPPORTED;
+  p.xr = 128;
+  p.wn = n;
+  p.n_mma = n;
+  p.a_rows = 128;
+  p.b_rows = n;
+  p.idesc = make_idesc(128, n, false, false);
+  if (!finish_plan(p, 3)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapA[0], dG, q, 128) || !map_kmajor(&p.mapA[1], dU, q, 128)) return AAL_ERR_UNSUPPORTED;
+  if (!map_kmajor(&p.mapB[0], Wg, 1, n) || !map_kmajor(&p.mapB[1], Wu, 1, n)) return AAL_ERR_UNSUPPORTED;
+  if (!out_map(p, dX, q)) return AAL_ERR_UNSUPPORTED;
+  p.n1 = (int)((p.Mq + 127) / 128);
+  p.n2 = q;
+  p.n3 = (int)(bi / n);
+  return launch<false, false, 3>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
 }
 
 aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
