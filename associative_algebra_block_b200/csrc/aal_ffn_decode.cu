@@ -201,7 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ffn_decode(const __grid_constan
   const bool up = (int)blockIdx.x < p.p1;  // gate/up CTA, else down CTA
   const int nops = up ? 2 : 1;
   const int K = up ? p.D : p.F;              // input rows of this CTA's projection
-  const int bi = K / p.q;                    // input group size
   const int bo = (up ? p.F : p.D) / p.q;     // output group size
   const int c0 = (up ? (int)blockIdx.x : (int)blockIdx.x - p.p1) * kCols;
   const int k = c0 / bo;                     // output group of the CTA's columns

@@ -142,6 +142,7 @@ struct Params {
   // arrives on, so the bounded wait runs out (after kStallNs), the kernel
   // records AAL_ERR_DEVICE_TIMEOUT and takes its abort path.
   int test_stall;
+  int map_mask;        // tensor maps in use: bits 0-1 mapA, 2-3 mapB, 4 mapOut
   // Segment mode (forward ops with explicit or ragged row types): the rows
   // were gathered type by type into contiguous segments; tile j of the device
   // table seg_tiles (j < *seg_count) is {type, first row, end of its type's
@@ -587,8 +588,14 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     }
     case OP_DX: {  // i0 class, i1 token block, i2 input group a, i3 column block of group a
       const int c = i0, a = i2, t = type_of_class(p, c);
-      for (int k = 0; k < p.q; ++k)
-        if (in_table(p.law, t, k, a)) add_seg(d, k * p.bo, p.bo, c, 0);
+      if (p.law == AAL_LAW_Q) {
+        // a in S(t, k) for Q_q: a == t (every k: one run over all groups) or k == a
+        if (a == t) add_seg(d, 0, p.q * p.bo, c, 0);
+        else add_seg(d, a * p.bo, p.bo, c, 0);
+      } else {
+        for (int k = 0; k < p.q; ++k)
+          if (in_table(p.law, t, k, a)) add_seg(d, k * p.bo, p.bo, c, 0);
+      }
       d.a_f = i1 * 128; d.a_c1 = 1;
       d.b_f = a * p.bi + i3 * p.wn; d.b_c1 = 0;
       d.rbase = i1 * 128; d.rstride = p.qv; d.roff = c; d.rlimit = p.Mq;
@@ -600,6 +607,10 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
       const int mb = p.swap ? i3 : i1, nb = p.swap ? i1 : i3;
       if (p.law == AAL_LAW_Q && a == k) {
         add_seg(d, 0, (int)p.Mall, 0, 1);  // every type uses the diagonal block
+      } else if (p.law == AAL_LAW_Q) {
+        // a != k: a in S(t, k) only for t == a, the class whose type is a
+        const int c = (a - p.off + p.q) % p.q;
+        if (c < p.qv) add_seg(d, 0, (int)p.Mq, c, 0);
       } else {
         for (int c = 0; c < p.qv; ++c)
           if (in_table(p.law, type_of_class(p, c), k, a)) add_seg(d, 0, (int)p.Mq, c, 0);
@@ -674,6 +685,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t smem0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   const int S = p.stages;
+  // Programmatic dependent launch: the next kernel of the stream may start
+  // its own set-up on SMs this grid has left; it reads nothing of ours before
+  // its griddepcontrol.wait, which returns once this grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;");
+  // start fetching the tensor maps in use while the barriers are set up
+  if (warp == kSchedWarp && lane < 5 && ((p.map_mask >> lane) & 1)) {
+    const CUtensorMap* m = lane < 2 ? &p.mapA[lane] : (lane < 4 ? &p.mapB[lane - 2] : &p.mapOut);
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(m)) : "memory");
+  }
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const bool issuer = !PAIR || rank == 0;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
@@ -718,6 +738,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   if (PAIR) cluster_sync_all();  // the peer's barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = s_tmem;
+  // Everything above touches only this CTA's shared memory, TMEM and its
+  // parameters; global memory (inputs a previous kernel of the stream writes,
+  // outputs it may still read) is used only after the previous grid is done.
+  // The tile decoder reads only parameters and shared memory (outside segment
+  // mode, whose tables are device data), so it describes the first tiles
+  // while a previous grid may still run.
+  if (warp != kSchedWarp || p.seg_mode) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0 || (warp >= 2 + kEpiWarps && warp < kSchedWarp)) {
     // ------------------------------------------------------ TMA producers
@@ -729,9 +756,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     const int pw = warp == 0 ? 0 : warp - (1 + kEpiWarps);
     uint32_t it = 0, st = 0, ph = 0, ti = 0;
     bool ok = pw < nprod;
-    for (int ss = tile0; tile_at(p, ss) >= 0 && ok; ss += tstep, ++ti) {
+    for (; ok; ++ti) {
       TileDesc d;
       if (!take_tile<true>(s_tile, tile_full, tile_empty, ti, d, &s_abort)) break;
+      if (d.nseg < 0) break;  // the decoder's end mark
       for (int s = 0; s < d.nseg && ok; ++s) {
         const Seg sg = seg_at(d, s);
         const int nch = seg_chunks(sg);
@@ -849,9 +877,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
       // test hook: a wait nothing ends, bounded by kStallNs; it records the
       // timeout and aborts the kernel before the first MMA
       if (p.test_stall && !mbar_wait(&stall_bar, 0, &s_abort, kStallNs)) ok = false;
-      for (int ss = tile0; tile_at(p, ss) >= 0 && ok; ss += tstep, ++tl) {
+      for (; ok; ++tl) {
         TileDesc d;
         if (!take_tile<false>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
+        if (d.nseg < 0) break;
         const uint32_t buf = tl & 1u, use = tl >> 1;
         if (!(mbar_try_wait(&tempty_bar[buf], (use & 1u) ^ 1u) ||
               mbar_wait(&tempty_bar[buf], (use & 1u) ^ 1u, &s_abort))) { ok = false; break; }
@@ -928,9 +957,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     uint32_t nstore = 0;
     uint32_t tl = 0;
     const int erow = PAIR ? (int)rank * 128 : 0;  // this CTA's 128 rows of the pair's tile
-    for (int ss = tile0; tile_at(p, ss) >= 0; ss += tstep, ++tl) {
+    for (;; ++tl) {
       TileDesc d;
       if (!take_tile<true>(s_tile, tile_full, tile_empty, tl, d, &s_abort)) break;
+      if (d.nseg < 0) break;
       d.rbase += erow;
       const uint32_t buf = tl & 1u, use = tl >> 1;
       if (!warp_wait(&tfull_bar[buf], use & 1u, &s_abort)) break;
@@ -1125,19 +1155,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     __syncwarp();
   } else if (warp == kSchedWarp) {
     // ------------------------------------------------------ tile decoder
+    // The only role that walks the schedule: the others take descriptions
+    // from the ring until the end mark (nseg = -1) that follows the last tile.
     if (lane == 0) {
       uint32_t i = 0;
       for (int ss = tile0; ; ss += tstep, ++i) {
         const int tile = tile_at(p, ss);
-        if (tile < 0) break;
         const uint32_t slot = i % kTileRing, ph = (i / kTileRing) & 1u;
         if (!(mbar_try_wait(&tile_empty[slot], ph ^ 1u) ||
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
           break;
         TileDesc d;
-        describe(p, tile, d);
+        if (tile >= 0) describe(p, tile, d);
+        else d.nseg = -1;
         s_tile[slot] = d;
         mbar_arrive(&tile_full[slot]);  // release: the copy above is visible first
+        if (tile < 0) break;
       }
     }
     __syncwarp();
@@ -1447,6 +1480,14 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (ntiles > INT_MAX) return AAL_ERR_UNSUPPORTED;
   p.ntiles = (int)ntiles;
   p.test_stall = test_stall_enabled();
+  p.map_mask = 0;
+  const CUtensorMap* maps[5] = {&p.mapA[0], &p.mapA[1], &p.mapB[0], &p.mapB[1], &p.mapOut};
+  for (int i = 0; i < 5; ++i) {
+    const unsigned char* b = reinterpret_cast<const unsigned char*>(maps[i]);
+    bool used = false;
+    for (size_t j = 0; j < sizeof(CUtensorMap) && !used; ++j) used = b[j] != 0;
+    if (used) p.map_mask |= 1 << i;
+  }
   if (!p.seg_mode) order_pairs(p);
   p.div_n1 = make_fastdiv((uint32_t)p.n1);
   p.div_n3 = make_fastdiv((uint32_t)p.n3);
@@ -1465,27 +1506,33 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
     attr_set |= bit;
   }
   const int sms = num_sms();
+  // every launch may overlap its set-up with the previous kernel's last CTAs
+  // (programmatic stream serialization; the kernel waits before any global access)
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     if (!p.seg_mode) schedule_tiles(p, grid);
     else p.use_order = 0;
-    k_tc<A_MN, B_MN, DUAL, false><<<grid, kThreads, smem, s>>>(p);
+    cfg.gridDim = dim3((unsigned)grid);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false>, p);
     note_launch();
-    return cuda_status(cudaGetLastError());
+    return cuda_status(e);
   }
   const int pairs = (int)(ntiles < sms / 2 ? ntiles : sms / 2);
-  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, true>, p);
   note_launch();
   return cuda_status(e);
