@@ -34,7 +34,7 @@ LAW = {"Q": 0, "Q2xQ2": 1}
 AAL_BF16, AAL_F32 = 0, 1
 AAL_TYPES_POSITION, AAL_TYPES_EXPLICIT = 0, 1
 AAL_PATH_AUTO, AAL_PATH_TENSOR, AAL_PATH_GENERAL, AAL_PATH_DECODE = 0, 1, 2, 3
-AAL_CALL_PROJECT_FWD, AAL_CALL_SWIGLU_FWD = 1, 2
+AAL_CALL_PROJECT_FWD, AAL_CALL_SWIGLU_FWD, AAL_CALL_PROJECT_BWD, AAL_CALL_SWIGLU_BWD = 1, 2, 3, 4
 
 EXPORTS = ("aal_project_fwd", "aal_swiglu_fwd", "aal_project_bwd", "aal_decode_matvec",
            "aal_swiglu_decode", "aal_swiglu_bwd", "aal_square_product", "aal_block_table", "aal_block_product_count",
@@ -303,8 +303,9 @@ def aal_set_timing_events(kernel: int, before=None, after=None):
 
 
 def aal_workspace_size(call, law, q, rule, rows, d_in, d_hidden=0) -> int:
-    """Bytes of device workspace the call needs for explicit or ragged row
-    types (0: none needed)."""
+    """Bytes of device workspace the call uses: the forward calls for explicit
+    or ragged row types, the backward calls to split their heavy Q_q tiles
+    (0: none used)."""
     n = int(load().aal_workspace_size(int(call), _law(law), q, rule, int(rows), int(d_in), int(d_hidden)))
     if n < 0:
         raise ValueError("aal_workspace_size: invalid arguments")

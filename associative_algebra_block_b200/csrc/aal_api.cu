@@ -88,6 +88,11 @@ static aal_status dispatch(int kind, cudaStream_t s, TC tc_launch, GEN gen_launc
   return st;
 }
 
+void* current_workspace(uint64_t* bytes) {
+  *bytes = t_ws_bytes;
+  return t_ws;
+}
+
 }  // namespace aal
 
 using namespace aal;
@@ -438,11 +443,20 @@ aal_status aal_set_timing_events(int32_t kernel, void* before, void* after) {
 int64_t aal_workspace_size(int32_t call, int32_t law, int32_t q, aal_row_type_rule rule, int64_t rows,
                            int64_t d_in, int64_t d_hidden) {
   if (!valid_law(law, q) || rows < 0 || d_in < 0 || d_hidden < 0 || !valid_rule(rule, rows)) return -1;
-  if (call != AAL_CALL_PROJECT_FWD && call != AAL_CALL_SWIGLU_FWD) return -1;
+  if (call < AAL_CALL_PROJECT_FWD || call > AAL_CALL_SWIGLU_BWD) return -1;
   const RowTypes rt = make_types(rule, q);
-  if (rows == 0 || !seg_needed(rt, q, rows)) return 0;
+  if (rows == 0) return 0;
+  if (call == AAL_CALL_PROJECT_BWD || call == AAL_CALL_SWIGLU_BWD) {
+    // split K of the heavy tiles (position rules on the tensor-core path only)
+    if (seg_needed(rt, q, rows)) return 0;
+    const int64_t a = tc_bwd_split_bytes(law, q, rows, d_in, d_hidden);
+    const int64_t b = call == AAL_CALL_SWIGLU_BWD ? tc_bwd_split_bytes(law, q, rows, d_hidden, d_in) : 0;
+    return a > b ? a : b;
+  }
+  if (!seg_needed(rt, q, rows)) return 0;
   return seg_workspace_bytes(q, rows, d_in, call == AAL_CALL_SWIGLU_FWD ? d_hidden : 0);
 }
+
 
 aal_status aal_set_workspace(void* device_ptr, uint64_t bytes) {
   if (device_ptr && ((uintptr_t)device_ptr % 256) != 0) return AAL_ERR_ALIGNMENT;

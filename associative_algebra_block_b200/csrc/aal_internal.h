@@ -129,6 +129,11 @@ aal_status tc_project_seg(int law, int q, long long rows, const aal_mat& Xg, con
 
 // ------------------------------------------- explicit / ragged row types
 bool seg_needed(const RowTypes& rt, int q, long long rows);
+// The caller's workspace of this host thread (aal_set_workspace), or null.
+void* current_workspace(uint64_t* bytes);
+// Workspace bytes the tensor-core backward of a projection W [din, dout]
+// uses to split its heavy Q_q tiles (0: no split for these sizes).
+int64_t tc_bwd_split_bytes(int law, int q, long long rows, long long din, long long dout);
 int64_t seg_workspace_bytes(int q, long long rows, long long w1, long long w2);
 aal_status seg_project_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& W,
                            const aal_mat& Y, void* ws, uint64_t ws_bytes, cudaStream_t s);

@@ -143,6 +143,15 @@ struct Params {
   // records AAL_ERR_DEVICE_TIMEOUT and takes its abort path.
   int test_stall;
   int map_mask;        // tensor maps in use: bits 0-1 mapA, 2-3 mapB, 4 mapOut
+  // Split K of the heavy Q_q tiles (dW diagonal blocks a == k, whose K runs
+  // over every token, and dX tiles a == t, whose K runs over every output
+  // group).  Heavy tile dg = (i0 * n1 + i1) * n3 + i3 is cut into ksplit
+  // pieces of split_len K positions: piece 0 is the tile's own slot, pieces
+  // 1.. are the extra tiles split_base + dg * (ksplit - 1) + piece - 1.  Each
+  // piece writes its fp32 accumulator to split_ws[dg * ksplit + piece][128][n_mma]
+  // (TMEM lane, column) and a reduction kernel adds the pieces.
+  int ksplit, split_len, split_base;
+  float* split_ws;
   // Segment mode (forward ops with explicit or ragged row types): the rows
   // were gathered type by type into contiguous segments; tile j of the device
   // table seg_tiles (j < *seg_count) is {type, first row, end of its type's
@@ -183,6 +192,7 @@ struct TileDesc {
   long long rlimit;
   long long cbase;
   int vlo, vhi;    // tile columns the epilogue writes (ragged mode)
+  int split;       // >= 0: a piece of a split heavy tile (partial-sum slot), else -1
 };
 
 // ------------------------------------------------------------------ PTX glue
@@ -525,16 +535,27 @@ __device__ __forceinline__ void describe_seg(const Params& p, int tile, TileDesc
 
 // tile = (pair_rank * n1 + i1) * n3 + i3; the pair is (i0, i2) of the op.
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
+  d.split = -1;
   if (p.seg_mode) {
     describe_seg(p, tile, d);
     return;
   }
-  const int t3 = (int)fdiv((uint32_t)tile, p.div_n3);
-  const int i3 = tile - t3 * p.n3;
-  const int pr = (int)fdiv((uint32_t)t3, p.div_n1);
-  const int i1 = t3 - pr * p.n1;
-  int i0, i2;
-  pair_of(p, pr, i0, i2);
+  int i0, i1, i2, i3, piece = 0;
+  if (p.ksplit > 1 && tile >= p.split_base) {
+    // an extra piece of heavy tile dg
+    const int j = tile - p.split_base, dg = j / (p.ksplit - 1);
+    piece = 1 + (j - dg * (p.ksplit - 1));
+    i3 = dg % p.n3;
+    i1 = (dg / p.n3) % p.n1;
+    i0 = dg / (p.n3 * p.n1);
+    i2 = p.op == OP_DW ? i0 : type_of_class(p, i0);
+  } else {
+    const int t3 = (int)fdiv((uint32_t)tile, p.div_n3);
+    i3 = tile - t3 * p.n3;
+    const int pr = (int)fdiv((uint32_t)t3, p.div_n1);
+    i1 = t3 - pr * p.n1;
+    pair_of(p, pr, i0, i2);
+  }
   d.nseg = 0;
   d.rstride = 1;
   d.roff = 0;
@@ -590,8 +611,15 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
       const int c = i0, a = i2, t = type_of_class(p, c);
       if (p.law == AAL_LAW_Q) {
         // a in S(t, k) for Q_q: a == t (every k: one run over all groups) or k == a
-        if (a == t) add_seg(d, 0, p.q * p.bo, c, 0);
-        else add_seg(d, a * p.bo, p.bo, c, 0);
+        if (a == t && p.ksplit > 1) {
+          const int k0 = piece * p.split_len;
+          add_seg(d, k0, min(p.split_len, p.q * p.bo - k0), c, 0);
+          d.split = ((c * p.n1 + i1) * p.n3 + i3) * p.ksplit + piece;
+        } else if (a == t) {
+          add_seg(d, 0, p.q * p.bo, c, 0);
+        } else {
+          add_seg(d, a * p.bo, p.bo, c, 0);
+        }
       } else {
         for (int k = 0; k < p.q; ++k)
           if (in_table(p.law, t, k, a)) add_seg(d, k * p.bo, p.bo, c, 0);
@@ -605,7 +633,11 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     case OP_DW: {  // i0 group a, i2 group k; (i1, i3) = (row slab, column block) or swapped
       const int a = i0, k = i2;
       const int mb = p.swap ? i3 : i1, nb = p.swap ? i1 : i3;
-      if (p.law == AAL_LAW_Q && a == k) {
+      if (p.law == AAL_LAW_Q && a == k && p.ksplit > 1) {
+        const int k0 = piece * p.split_len;
+        add_seg(d, k0, (int)min((long long)p.split_len, p.Mall - k0), 0, 1);
+        d.split = ((a * p.n1 + i1) * p.n3 + i3) * p.ksplit + piece;
+      } else if (p.law == AAL_LAW_Q && a == k) {
         add_seg(d, 0, (int)p.Mall, 0, 1);  // every type uses the diagonal block
       } else if (p.law == AAL_LAW_Q) {
         // a != k: a in S(t, k) only for t == a, the class whose type is a
@@ -1000,6 +1032,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             if (PAIR) mbar_arrive_remote(tempty_addr);
             else mbar_arrive(&tempty_bar[buf]);
           }
+        }
+        if (p.ksplit > 1 && d.split >= 0) {
+          // a piece of a split tile: its fp32 partial, TMEM lane by column
+          float4* dst = reinterpret_cast<float4*>(
+              p.split_ws + ((size_t)d.split * 128 + row_in_tile) * p.n_mma + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          continue;
         }
         if (p.tma_store && (c0 < d.vlo || c0 + 16 > d.vhi)) {
           // ragged mode: a chunk at or past the edge of the group's columns;
@@ -1438,11 +1478,18 @@ static void schedule_tiles(Params& p, int grid) {
   if (grid <= 0 || nt <= grid || nt > kMaxOrder) return;
   std::vector<int> cost(nt), idx(nt);
   const int per_pair = p.n1 * p.n3;
+  const bool split = p.ksplit > 1;
+  const int piece_cost = split ? (p.q + p.ksplit - 1) / p.ksplit : 0;
   for (int t = 0; t < nt; ++t) {
+    idx[t] = t;
+    if (split && t >= p.split_base) {  // an extra piece of a split heavy tile
+      cost[t] = piece_cost;
+      continue;
+    }
     int p0, p1;
     host_pair_of(p, t / per_pair, p0, p1);
     cost[t] = pair_cost(p, p0, p1);
-    idx[t] = t;
+    if (split && cost[t] == p.q) cost[t] = piece_cost;  // the heavy tile's own piece
   }
   std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
   std::vector<std::vector<int>> lists(grid);
@@ -1464,6 +1511,90 @@ static void schedule_tiles(Params& p, int grid) {
       p.order[r * grid + c] = r < lists[c].size() ? (uint16_t)lists[c][r] : (uint16_t)0xFFFF;
   p.nslots = (int)(rounds * grid);
   p.use_order = 1;
+}
+
+// ------------------------------------------------ split-K of the heavy tiles
+struct SplitReduce {
+  const float* ws;
+  __nv_bfloat16* out;
+  long long ldo, Mq;
+  int op, ksplit, n, nheavy, n1, n3, bi, bo, wn, swap, accumulate, q, off, qv;
+};
+
+// Adds the ksplit fp32 partials of every heavy tile and writes the bf16 result
+// (added to the output when accumulating): one thread per 4 columns of a TMEM
+// lane of a heavy tile.
+__global__ void __launch_bounds__(256) k_split_reduce(const SplitReduce r) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int nq = r.n >> 2;
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)r.nheavy * 128 * nq) return;
+  const int cq = (int)(gid % nq);
+  const long long rest = gid / nq;
+  const int lane = (int)(rest % 128);
+  const int dg = (int)(rest / 128);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < r.ksplit; ++s) {
+    const float4 v =
+        reinterpret_cast<const float4*>(r.ws + ((size_t)(dg * r.ksplit + s) * 128 + lane) * r.n)[cq];
+    acc[0] += v.x;
+    acc[1] += v.y;
+    acc[2] += v.z;
+    acc[3] += v.w;
+  }
+  const int i3 = dg % r.n3, i1 = (dg / r.n3) % r.n1, i0 = dg / (r.n3 * r.n1);
+  const int col = 4 * cq;
+  if (r.op == OP_DW) {
+    // block (a, a): TMEM lanes are rows of dW (columns when swapped)
+    const int a = i0, mb = r.swap ? i3 : i1, nb = r.swap ? i1 : i3;
+    const long long xf = (long long)a * r.bi + (r.swap ? (long long)nb * r.wn : (long long)mb * 128);
+    const long long yf = (long long)a * r.bo + (r.swap ? (long long)mb * 128 : (long long)nb * r.wn);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long long rr = r.swap ? xf + col + j : xf + lane;
+      const long long cc = r.swap ? yf + lane : yf + col + j;
+      __nv_bfloat16* o = r.out + rr * r.ldo + cc;
+      const float v = r.accumulate ? acc[j] + __bfloat162float(*o) : acc[j];
+      *o = __float2bfloat16_rn(v);
+    }
+  } else {
+    // dX tile (class c, group a = type of c): TMEM lanes are the class's rows
+    const int c = i0;
+    int t = c + r.off;
+    if (t >= r.q) t -= r.q;
+    const long long x = (long long)i1 * 128 + lane;
+    if (x >= r.Mq) return;
+    __nv_bfloat16* o = r.out + (x * r.qv + c) * r.ldo + (long long)t * r.bi + (long long)i3 * r.wn + col;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float v = r.accumulate ? acc[j] + __bfloat162float(o[j]) : acc[j];
+      o[j] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// Split factor of the heavy tiles: pieces of about the average load of a CTA
+// (counted in 64-wide K chunks), no smaller than a light tile.  The pieces'
+// partial sums go through the caller's workspace and a reduction kernel.
+static void plan_split(Params& p, long long heavy_k, long long light_k, long long nheavy,
+                       long long nlight) {
+  p.ksplit = 0;
+  if (nheavy <= 0 || heavy_k <= 64) return;
+  const long long ch = (heavy_k + 63) / 64, cl = (light_k + 63) / 64;
+  const long long grid = std::min<long long>(nheavy + nlight, num_sms());
+  const long long total = nheavy * ch + nlight * cl;
+  const long long target = std::max(cl, (total + grid - 1) / grid);
+  // the reduction costs about as much as 16 chunks of a heavy tile: split only
+  // tiles that run at least that much longer than a CTA's average load
+  if (ch - target < 16) return;
+  long long S = std::min<long long>((ch + target - 1) / target, 16);
+  if (S < 2) return;
+  const long long len = ((heavy_k + S - 1) / S + 63) / 64 * 64;
+  S = (heavy_k + len - 1) / len;
+  if (S < 2 || len > INT_MAX) return;
+  p.ksplit = (int)S;
+  p.split_len = (int)len;
 }
 
 // AAL_TEST_STALL=1 in the environment turns on Params::test_stall for the
@@ -1537,6 +1668,94 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   note_launch();
   return cuda_status(e);
 }
+
+// Launches the op with its heavy tiles split (when plan_split chose to and the
+// caller's workspace holds the partial sums) and the reduction of the pieces.
+template <bool A_MN, bool B_MN, int DUAL>
+static aal_status launch_split(Params& p, long long base_tiles, long long nheavy, cudaStream_t s) {
+  uint64_t have = 0;
+  float* ws = static_cast<float*>(current_workspace(&have));
+  const size_t bytes = p.ksplit > 1 ? (size_t)nheavy * p.ksplit * 128 * p.n_mma * sizeof(float) : 0;
+  if (p.ksplit < 2 || !ws || have < bytes) {
+    p.ksplit = 0;
+    return launch<A_MN, B_MN, DUAL>(p, base_tiles, s);
+  }
+  p.split_ws = ws;
+  p.split_base = (int)base_tiles;
+  aal_status st = launch<A_MN, B_MN, DUAL>(p, base_tiles + nheavy * (p.ksplit - 1), s);
+  if (st == AAL_OK) {
+    SplitReduce r;
+    r.ws = ws;
+    r.out = p.out;
+    r.ldo = p.ldo;
+    r.Mq = p.Mq;
+    r.op = p.op;
+    r.ksplit = p.ksplit;
+    r.n = p.n_mma;
+    r.nheavy = (int)nheavy;
+    r.n1 = p.n1;
+    r.n3 = p.n3;
+    r.bi = p.bi;
+    r.bo = p.bo;
+    r.wn = p.wn;
+    r.swap = p.swap;
+    r.accumulate = p.accumulate;
+    r.q = p.q;
+    r.off = p.off;
+    r.qv = p.qv;
+    const long long threads = nheavy * 128 * (p.n_mma / 4);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    st = cuda_status(cudaLaunchKernelEx(&cfg, k_split_reduce, r));
+    note_launch();
+  }
+  return st;
+}
+
+// Heavy-tile geometry of the dX and dW launches (kept in step with their planners).
+struct SplitGeom {
+  long long nheavy = 0, nlight = 0, heavy_k = 0, light_k = 0;
+  int n = 0;
+};
+static SplitGeom geom_dx(int q, long long rows, long long bi, long long bo) {
+  SplitGeom g;
+  g.n = pick_n(bi, 256);
+  if (!g.n) return g;
+  const long long n1 = (rows / q + 127) / 128, n3 = bi / g.n;
+  g.nheavy = (long long)q * n1 * n3;
+  g.nlight = (long long)q * n1 * q * n3 - g.nheavy;
+  g.heavy_k = (long long)q * bo;
+  g.light_k = bo;
+  return g;
+}
+static SplitGeom geom_dw(int q, long long rows, long long bi, long long bo) {
+  SplitGeom g;
+  const bool swap = bi % 128 != 0;
+  if (swap && bo % 128 != 0) return g;
+  g.n = pick_n(swap ? bi : bo, 256);
+  if (!g.n) return g;
+  const long long n1 = swap ? bi / g.n : bi / 128, n3 = swap ? bo / 128 : bo / g.n;
+  g.nheavy = (long long)q * n1 * n3;
+  g.nlight = (long long)q * n1 * q * n3 - g.nheavy;
+  g.heavy_k = rows;
+  g.light_k = rows / q;
+  return g;
+}
+static int64_t split_bytes(const SplitGeom& g) {
+  if (!g.n || g.nheavy <= 0) return 0;
+  Params p;
+  memset(&p, 0, sizeof(p));
+  plan_split(p, g.heavy_k, g.light_k, g.nheavy, g.nlight);
+  return p.ksplit > 1 ? (int64_t)g.nheavy * p.ksplit * 128 * g.n * (int64_t)sizeof(float) : 0;
+}
+
 
 // AAL_TC_PAIR=1 in the environment turns the CTA-pair mode on.  It is off by
 // default: on B200 the single-CTA kernel with four producer warps and the
@@ -1836,7 +2055,11 @@ static aal_status bwd_dx_impl(int law, int q, const RowTypes& rt, long long rows
   p.n1 = (int)((p.Mq + 127) / 128);
   p.n2 = q;
   p.n3 = (int)(bi / n);
-  return launch<false, false, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+  const long long base = (long long)q * p.n1 * p.n2 * p.n3, nheavy = (long long)q * p.n1 * p.n3;
+  // heavy tiles (a == t) run over all q output groups; the SiLU' epilogue needs
+  // the whole sum in one place, so the dH kernel keeps them whole
+  if (law == AAL_LAW_Q && q > 1 && !G) plan_split(p, (long long)q * bo, bo, nheavy, base - nheavy);
+  return launch_split<false, false, 0>(p, base, nheavy, s);
 }
 
 // dX of the SwiGLU backward in one launch: dX = dG Wg^T + dU Wu^T through the
@@ -1872,7 +2095,9 @@ aal_status tc_swiglu_bwd_dx(int law, int q, const RowTypes& rt, long long rows, 
   p.n1 = (int)((p.Mq + 127) / 128);
   p.n2 = q;
   p.n3 = (int)(bi / n);
-  return launch<false, false, 3>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+  const long long base = (long long)q * p.n1 * p.n2 * p.n3, nheavy = (long long)q * p.n1 * p.n3;
+  if (law == AAL_LAW_Q && q > 1) plan_split(p, (long long)q * bo, bo, nheavy, base - nheavy);
+  return launch_split<false, false, 3>(p, base, nheavy, s);
 }
 
 aal_status tc_project_bwd_dx(int law, int q, const RowTypes& rt, long long rows, const aal_mat& dY,
@@ -1884,6 +2109,14 @@ aal_status tc_swiglu_bwd_dh(int law, int q, const RowTypes& rt, long long rows, 
                             const aal_mat& Wd, const aal_mat& G, const aal_mat& U,
                             const aal_mat& dG, const aal_mat& dU, cudaStream_t s) {
   return bwd_dx_impl(law, q, rt, rows, dY, Wd, dG, 0, &G, &U, &dU, s);
+}
+
+int64_t tc_bwd_split_bytes(int law, int q, long long rows, long long din, long long dout) {
+  if (law != AAL_LAW_Q || q < 2 || rows % q || din % q || dout % q) return 0;
+  const long long bi = din / q, bo = dout / q;
+  if (bi % 16 || bo % 16) return 0;
+  const int64_t a = split_bytes(geom_dx(q, rows, bi, bo)), b = split_bytes(geom_dw(q, rows, bi, bo));
+  return a > b ? a : b;
 }
 
 aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,
@@ -1938,7 +2171,10 @@ aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows,
   if (!swap) { p.n1 = (int)(bi / 128); p.n3 = (int)(bo / n); }
   else { p.n1 = (int)(bi / n); p.n3 = (int)(bo / 128); }
   p.n2 = q;
-  return launch<true, true, 0>(p, (long long)q * p.n1 * p.n2 * p.n3, s);
+  const long long base = (long long)q * p.n1 * p.n2 * p.n3, nheavy = (long long)q * p.n1 * p.n3;
+  // heavy tiles: the diagonal blocks, whose K runs over every token
+  if (law == AAL_LAW_Q && q > 1) plan_split(p, rows, p.Mq, nheavy, base - nheavy);
+  return launch_split<true, true, 0>(p, base, nheavy, s);
 }
 
 aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const aal_mat& Z,

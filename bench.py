@@ -364,8 +364,10 @@ class ProjFwdBwd:
 
     def config(self):
         return {"workload": f"{self.name}: {self.law} q={self.q} projections {self.D}->{self.F} and "
-                            f"{self.F}->{self.D}, M={self.M}, fwd + bwd (dX, dW)",
-                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F}
+                            f"{self.F}->{self.D}, M={self.M}, fwd + bwd (dX, dW); heavy Q_q tiles "
+                            f"split through a workspace",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F,
+                "workspace_bytes": getattr(self, "ws_bytes", None)}
 
     def bytes_per_set(self):
         return 2 * (2 * self.D * self.F * 3 + self.M * (self.D + self.F) * 4)
@@ -384,6 +386,11 @@ class ProjFwdBwd:
                 s[tag + "dW"] = torch.empty_like(s[tag + "W"])
             self.sets.append(s)
         self.rule = aal.row_rule(seq_len=self.seq_len)
+        # workspace for the split of the heavy dX / dW tiles (the larger of the two shapes)
+        self.ws_bytes = max(aal.aal_workspace_size(aal.AAL_CALL_PROJECT_BWD, self.law, self.q, self.rule,
+                                                   self.M, a_, b_, ) for a_, b_ in ((self.D, self.F), (self.F, self.D)))
+        for s in self.sets:
+            s["ws"] = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device="cuda")
         s0 = self.sets[0]
         self.pin = dict(inp={t + k: s0[t + k].cpu().pin_memory() for t in "ab" for k in ("X", "dY")},
                         out=[{t + k: torch.empty_like(s0[t + k], device="cpu").pin_memory()
@@ -408,6 +415,7 @@ class ProjFwdBwd:
     def step(self, i, ev=None, gev=None):
         s = self.sets[i % len(self.sets)]
         mark = _marker(ev)
+        aal.aal_set_workspace(s["ws"])
         for n, t in enumerate(("a", "b")):
             mark(3 * n)
             aal.aal_project_fwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "Y"])
@@ -415,6 +423,7 @@ class ProjFwdBwd:
             mark(3 * n + 2)
             aal.aal_project_bwd(self.law, self.q, self.rule, s[t + "X"], s[t + "W"], s[t + "dY"],
                                 s[t + "dX"], s[t + "dW"])
+        aal.aal_set_workspace(None)
 
     def dense_step(self, i):
         s = self.sets[i % len(self.sets)]
@@ -482,8 +491,10 @@ class SwigluFwdBwd:
         return {"workload": f"{self.name}: {self.law} q={self.q} SwiGLU FFN D={self.D} F={self.F} "
                             f"M={self.M}, forward + backward (dX, dWg, dWu, dWd); executed FLOPs "
                             f"count the 9 row-typed products the chain rule needs, not the "
-                            f"recomputed G and U",
-                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F}
+                            f"recomputed G and U; heavy Q_q tiles of the backward split through a "
+                            f"workspace",
+                "law": self.law, "q": self.q, "M": self.M, "d": self.D, "ffn": self.F,
+                "workspace_bytes": getattr(self, "ws_bytes", None)}
 
     def bytes_per_set(self):
         e = 2
@@ -506,6 +517,10 @@ class SwigluFwdBwd:
             t["dWd"] = torch.empty(F, D, dtype=torch.bfloat16, device="cuda")
             self.sets.append(t)
         self.rule = aal.row_rule(seq_len=self.seq_len)
+        # workspace for the split of the backward's heavy tiles
+        self.ws_bytes = aal.aal_workspace_size(aal.AAL_CALL_SWIGLU_BWD, self.law, self.q, self.rule, M, D, F)
+        for t in self.sets:
+            t["ws"] = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device="cuda")
         s0 = self.sets[0]
         self.pin = dict(inp={k: s0[k].cpu().pin_memory() for k in ("X", "dY")},
                         out=[{k: torch.empty_like(s0[k], device="cpu").pin_memory()
@@ -538,8 +553,10 @@ class SwigluFwdBwd:
         aal.aal_swiglu_fwd(self.law, self.q, self.rule, t["X"], t["Wg"], t["Wu"], t["Wd"], t["H"], t["Y"])
         for j in range(2, 6):
             mark(j)
+        aal.aal_set_workspace(t["ws"])
         aal.aal_swiglu_bwd(self.law, self.q, self.rule, t["X"], t["Wg"], t["Wu"], t["Wd"], t["H"], t["dY"],
                            t["G"], t["U"], t["dG"], t["dU"], t["dX"], t["dWg"], t["dWu"], t["dWd"])
+        aal.aal_set_workspace(None)
 
     def dense_step(self, i):
         """Dense SwiGLU forward and backward with the same products:

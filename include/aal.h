@@ -270,10 +270,22 @@ AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat
  * AAL_ERR_UNSUPPORTED).  The backward calls always take the general path for
  * such rules.
  *
+ * The backward calls use a workspace differently: under Q_q a few tiles are
+ * far longer than the rest (the diagonal blocks of dW sum over every token;
+ * the dX blocks a == t sum over every output group), and with a large enough
+ * workspace aal_project_bwd and aal_swiglu_bwd cut those tiles into K pieces
+ * that run on separate SMs, keep the pieces' fp32 partial sums in the
+ * workspace and add them in a short reduction kernel.  The result is the
+ * same sum in another association order.  The dH step of aal_swiglu_bwd
+ * (its SiLU' chain needs the whole sum) is never split.
+ *
  * aal_workspace_size: bytes the call needs for ``rows`` rows; call is
- * AAL_CALL_PROJECT_FWD (d_in = din, d_hidden unused) or AAL_CALL_SWIGLU_FWD
- * (d_in = D, d_hidden = F).  0 when the rule needs none, -1 for invalid
- * arguments.  Roughly rows * (d_in [+ d_hidden]) * 2 + rows * 4 bytes.
+ * AAL_CALL_PROJECT_FWD (d_in = din, d_hidden unused), AAL_CALL_SWIGLU_FWD
+ * (d_in = D, d_hidden = F), AAL_CALL_PROJECT_BWD (d_in = din, d_hidden =
+ * dout) or AAL_CALL_SWIGLU_BWD (d_in = D, d_hidden = F).  0 when the call
+ * uses none, -1 for invalid arguments.  Forward: roughly rows * (d_in
+ * [+ d_hidden]) * 2 + rows * 4 bytes; backward: the heavy tiles' partial
+ * sums (e.g. 17 MB for M = 2048, din = 2048, dout = 768, q = 16).
  *
  * aal_set_workspace: device memory the following calls of this host thread
  * may use (NULL or 0 bytes: none).  The pointer must be 256-byte aligned
@@ -283,7 +295,8 @@ AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat
  * share a workspace.  Supported: bf16, q <= 256, 16-byte aligned rows,
  * din / q and dout / q multiples of 16.
  */
-enum { AAL_CALL_PROJECT_FWD = 1, AAL_CALL_SWIGLU_FWD = 2 };
+enum { AAL_CALL_PROJECT_FWD = 1, AAL_CALL_SWIGLU_FWD = 2, AAL_CALL_PROJECT_BWD = 3,
+       AAL_CALL_SWIGLU_BWD = 4 };
 AAL_API int64_t aal_workspace_size(int32_t call, int32_t law, int32_t q, aal_row_type_rule rule,
                            int64_t rows, int64_t d_in, int64_t d_hidden);
 AAL_API aal_status aal_set_workspace(void* device_ptr, uint64_t bytes);

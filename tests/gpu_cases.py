@@ -134,7 +134,7 @@ def run_swiglu(law, q, M, D, F, dtype, seq_len, w_sigma_rule="din", seed=0,
 
 
 def run_bwd(law, q, M, din, dout, dtype, seq_len=None, explicit=False, seed=0, accumulate=False,
-            policy=aal.AAL_PATH_AUTO):
+            policy=aal.AAL_PATH_AUTO, ws=False):
     ins = inputs.projection_inputs(M, din, dout, seed=seed, dtype=dtype, with_dy=True)
     X, W, dY = dev(ins["X"]), dev(ins["W"]), dev(ins["dY"])
     dX = torch.full((M, din), float("nan"), dtype=X.dtype, device="cuda")
@@ -154,11 +154,18 @@ def run_bwd(law, q, M, din, dout, dtype, seq_len=None, explicit=False, seed=0, a
         types = packed_types(law, q, M, seq_len)
     aal.aal_set_path_policy(policy)
     try:
-        aal.aal_project_bwd(law, q, rule, X, W, dY, dX, dW, accumulate_dW=accumulate)
-        torch.cuda.synchronize()
+        if ws:
+            with workspace(aal.AAL_CALL_PROJECT_BWD, law, q, rule, M, din, dout) as w:
+                assert w.n > 0
+                aal.aal_project_bwd(law, q, rule, X, W, dY, dX, dW, accumulate_dW=accumulate)
+                torch.cuda.synchronize()
+        else:
+            aal.aal_project_bwd(law, q, rule, X, W, dY, dX, dW, accumulate_dW=accumulate)
+            torch.cuda.synchronize()
         path = aal.aal_last_path()
     finally:
         aal.aal_set_path_policy(aal.AAL_PATH_AUTO)
+    assert aal.aal_get_device_status() == aal.AAL_OK
     rdX, rdW = oracle.project_bwd(law, q, types, ins["X"].f64, ins["W"].f64, ins["dY"].f64)
     if base is not None:
         rdW = rdW + base.f64
@@ -206,7 +213,7 @@ def run_swiglu_decode(law, q, B, D, F, dtype, seq_len=1536, seed=0, same_type=No
 
 
 def run_swiglu_bwd(law, q, M, D, F, dtype, seq_len=None, seed=0, explicit=False,
-                   policy=aal.AAL_PATH_AUTO):
+                   policy=aal.AAL_PATH_AUTO, ws=False):
     ins = inputs.swiglu_inputs(D, F, M, seed=seed, dtype=dtype)
     X, Wg, Wu, Wd = (dev(ins[k]) for k in ("X", "Wg", "Wu", "Wd"))
     dYd = inputs.Stream(seed + 7).normal(M, D, 1.0, dtype)
@@ -225,10 +232,16 @@ def run_swiglu_bwd(law, q, M, D, F, dtype, seq_len=None, seed=0, explicit=False,
     aal.aal_set_path_policy(policy)
     try:
         aal.aal_swiglu_fwd(law, q, rule, X, Wg, Wu, Wd, H, Y)
-        ws = [torch.full((M, F), float("nan"), dtype=X.dtype, device="cuda") for _ in range(4)]
+        hs = [torch.full((M, F), float("nan"), dtype=X.dtype, device="cuda") for _ in range(4)]
         outs = [torch.full(t.shape, float("nan"), dtype=X.dtype, device="cuda") for t in (X, Wg, Wu, Wd)]
-        aal.aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, *ws, *outs)
-        torch.cuda.synchronize()
+        if ws:
+            with workspace(aal.AAL_CALL_SWIGLU_BWD, law, q, rule, M, D, F) as w:
+                assert w.n > 0
+                aal.aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, *hs, *outs)
+                torch.cuda.synchronize()
+        else:
+            aal.aal_swiglu_bwd(law, q, rule, X, Wg, Wu, Wd, H, dY, *hs, *outs)
+            torch.cuda.synchronize()
         path = aal.aal_last_path()
     finally:
         aal.aal_set_path_policy(aal.AAL_PATH_AUTO)

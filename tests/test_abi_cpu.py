@@ -264,3 +264,19 @@ def test_every_compute_binding_runs_an_empty_call(lib):
     assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_FWD, "Q", 2, rule, 0, 8) == 0
     assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_FWD, "Q", 2, aal.row_rule(seq_len=7), 10, 64) > 10 * 64 * 2
     aal.aal_set_workspace(None)
+
+
+def test_backward_workspace_sizes():
+    # the backward calls use a workspace for the split of their heavy Q_q tiles
+    rule = aal.row_rule(seq_len=2048)
+    n = aal.aal_workspace_size(aal.AAL_CALL_PROJECT_BWD, "Q", 16, rule, 2048, 2048, 768)
+    assert n > 0 and n % (128 * 4) == 0
+    assert aal.aal_workspace_size(aal.AAL_CALL_SWIGLU_BWD, "Q", 16, rule, 2048, 2048, 768) >= n
+    # no heavy tiles to split: the Q2xQ2 law, q = 1
+    assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_BWD, "Q2xQ2", 4, rule, 2048, 768, 1536) == 0
+    assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_BWD, "Q", 1, rule, 2048, 2048, 768) == 0
+    # rules that take the general path use none
+    assert aal.aal_workspace_size(aal.AAL_CALL_PROJECT_BWD, "Q", 16, aal.row_rule(seq_len=7), 2048,
+                                  2048, 768) == 0
+    with pytest.raises(ValueError):
+        aal.aal_workspace_size(5, "Q", 16, rule, 2048, 2048, 768)

@@ -266,10 +266,12 @@ def test_c3_projection_full_size():
 
 # ------------------------------------------ Qwen3-30B-A3B-expert-shaped Q_16
 @pytest.mark.parametrize("din,dout", [(2048, 768), (768, 2048)])
-def test_c4_projection_fwd_bwd(din, dout):
+@pytest.mark.parametrize("ws", [False, True])
+def test_c4_projection_fwd_bwd(din, dout, ws):
+    # ws: with a workspace the heavy dX / dW tiles run as split K pieces
     err, path = run_project("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
     assert err <= TOL["bf16"] and path == TENSOR, err
-    edx, edw, path = run_bwd("Q", 16, 2048, din, dout, "bf16", seq_len=2048)
+    edx, edw, path = run_bwd("Q", 16, 2048, din, dout, "bf16", seq_len=2048, ws=ws)
     assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
     assert path == TENSOR
 
@@ -383,9 +385,29 @@ def test_q1_is_dense():
     assert err <= TOL["bf16"], err
 
 
-def test_bwd_accumulate():
-    edx, edw, _ = run_bwd("Q", 4, 512, 256, 256, "bf16", accumulate=True)
+@pytest.mark.parametrize("q,M,din,dout,ws", [(4, 512, 256, 256, False), (8, 1600, 3072, 256, True)])
+def test_bwd_accumulate(q, M, din, dout, ws):
+    # dW += X^T dY; with ws the diagonal blocks are split and their reduction adds to dW
+    edx, edw, _ = run_bwd("Q", q, M, din, dout, "bf16", seq_len=M, accumulate=True, ws=ws)
     assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
+
+
+def test_bwd_split_heavy_tiles_ragged_rows():
+    # Q_8 with 200 rows per class (a partial 128-row block) and two column
+    # blocks per input group: the heavy dX tiles (a == t, K over every output
+    # group) and dW tiles (diagonal blocks, K over every token) run as K pieces
+    # whose fp32 partials a reduction kernel adds
+    edx, edw, path = run_bwd("Q", 8, 1600, 3072, 256, "bf16", seq_len=1600, ws=True)
+    assert edx <= TOL["bf16"] and edw <= TOL["bf16"], (edx, edw)
+    assert path == TENSOR
+
+
+def test_swiglu_bwd_split_heavy_tiles():
+    # expert shape with a workspace: dX (both products in one accumulator),
+    # dWg, dWu and dWd split their heavy tiles; dH keeps them whole
+    errs, got = run_swiglu_bwd("Q", 16, 2048, 2048, 768, "bf16", seed=5, ws=True)
+    assert max(errs) <= TOL["bf16"], errs
+    assert got == TENSOR
 
 
 def test_general_path_matches_oracle():
