@@ -59,6 +59,7 @@ constexpr int kTileRing = 8;
 // processing time first onto the least loaded CTA) and passed with the launch.
 constexpr int kMaxOrder = 1024;
 constexpr int kMaxPairs = 256;
+constexpr int kMaxSegs = 6;  // K segments of one tile
 constexpr int kMaxStages = 8;
 constexpr int kSmemBudget = 224 * 1024;  // + 1 KB alignment slack, under the 227 KB per-CTA limit
 constexpr int kEpiSmem = kEpiWarps * 2048;  // TMA-store staging
@@ -152,6 +153,12 @@ struct Params {
   // (TMEM lane, column) and a reduction kernel adds the pieces.
   int ksplit, split_len, split_base;
   float* split_ws;
+  // Class-group mode (swapped forward under Q_q): a tile covers grp classes
+  // of grp_n token rows each; its diagonal segment is one MMA over all of them
+  // (N = grp * grp_n, idesc), its per-class segments MMAs of N = grp_n
+  // (idesc_one) into the class's TMEM columns.  box_bytes: one class's B box.
+  int grp, grp_n;
+  uint32_t idesc_one, box_bytes;
   // Segment mode (forward ops with explicit or ragged row types): the rows
   // were gathered type by type into contiguous segments; tile j of the device
   // table seg_tiles (j < *seg_count) is {type, first row, end of its type's
@@ -183,7 +190,7 @@ struct Params {
 static_assert(sizeof(Params) <= 4096, "kernel parameters stay within the classic 4 KB limit");
 
 struct TileDesc {
-  Seg seg[4];
+  Seg seg[kMaxSegs];
   int nseg;
   int a_f, b_f;    // fixed coordinate of A / B (row start of K-major, column start of MN-major)
   int a_c1, b_c1;  // 1: coordinate 1 is the segment's class
@@ -430,7 +437,7 @@ __device__ __forceinline__ void add_seg(TileDesc& d, int k0, int len, int cls, i
   // merge with the previous segment when the K ranges touch (same class/map)
   bool merged = false;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < kMaxSegs; ++j) {
     Seg& s = d.seg[j];
     if (j == d.nseg - 1 && s.cls == cls && s.map == map && s.k0 + s.len == k0) {
       s.len += len;
@@ -439,7 +446,7 @@ __device__ __forceinline__ void add_seg(TileDesc& d, int k0, int len, int cls, i
   }
   if (merged) return;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
+  for (int j = 0; j < kMaxSegs; ++j) {
     if (j == d.nseg) {
       d.seg[j].k0 = k0;
       d.seg[j].len = len;
@@ -454,6 +461,8 @@ __device__ __forceinline__ Seg seg_at(const TileDesc& d, int s) {
   if (s == 1) r = d.seg[1];
   if (s == 2) r = d.seg[2];
   if (s == 3) r = d.seg[3];
+  if (s == 4) r = d.seg[4];
+  if (s == 5) r = d.seg[5];
   return r;
 }
 // The members a of S(t, k) in ascending order, each added as a K segment of
@@ -534,8 +543,39 @@ __device__ __forceinline__ void describe_seg(const Params& p, int tile, TileDesc
 }
 
 // tile = (pair_rank * n1 + i1) * n3 + i3; the pair is (i0, i2) of the op.
+// Class-group tile (cg, k, i3): classes c0 = cg * grp ... c0 + grp - 1, output
+// group k, 128-column block i3 of it.  Under Q_q every class's rows add
+// X_c[., k] W(k, k) (the diagonal term, one segment over all grp classes: B
+// is their boxes side by side) and, for type t(c) != k, X_c[., t] W(t, k)
+// (one segment per class, into that class's TMEM columns).
+__device__ __forceinline__ void describe_grp(const Params& p, int tile, TileDesc& d) {
+  const int i3 = tile % p.n3, r = tile / p.n3, k = r % p.q, cg = r / p.q;
+  const int c0 = cg * p.grp, wcol0 = k * p.bo + i3 * p.wn;
+  d.nseg = 0;
+  add_seg(d, k * p.bi, p.bi, c0, p.grp);
+  for (int j = 0; j < p.grp; ++j) {
+    const int c = c0 + j, t = type_of_class(p, c);
+    if (t != k) add_seg(d, t * p.bi, p.bi, c, 1);
+  }
+  d.a_f = wcol0;
+  d.a_c1 = 0;
+  d.b_f = 0;
+  d.b_c1 = 1;
+  d.rbase = 0;
+  d.rstride = p.qv;
+  d.roff = c0;
+  d.rlimit = p.Mq;
+  d.cbase = wcol0;
+  d.vlo = 0;
+  d.vhi = INT_MAX;
+}
+
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
   d.split = -1;
+  if (p.grp) {
+    describe_grp(p, tile, d);
+    return;
+  }
   if (p.seg_mode) {
     describe_seg(p, tile, d);
     return;
@@ -804,7 +844,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const uint32_t base = smem0 + st * p.stage_bytes;
             const int kofs = sg.k0 + kc * 64;
             const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
-            if (lane == 0 && issuer) mbar_expect_tx(&full_bar[st], (PAIR ? 2u : 1u) * p.tx_bytes);
+            if (lane == 0 && issuer) {
+              // class-group mode: the segment's classes' B boxes (sg.map of them)
+              const uint32_t tx = p.grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
+                                        : (PAIR ? 2u : 1u) * p.tx_bytes;
+              mbar_expect_tx(&full_bar[st], tx);
+            }
             if (lane == 0) atomicMax(&s_last_chunk[st], (int)it);
             if (!A_MN && B_MN && DUAL == 0 && !PAIR && p.ragged) {
               // lane 0: the A box; lane 1: the B box (all atoms, ka rows from -oa)
@@ -817,13 +862,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const int na = DUAL >= 2 ? 2 : 1;
             const int nb = ((DUAL == 1 && !PAIR) || DUAL == 3) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
-            const int nB = (B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1;  // boxes per B operand
+            const int nB = p.grp ? sg.map : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
             const int arow = PAIR ? (int)rank * 128 : 0;  // this CTA's half of the A tile
             const int bsh = (PAIR && DUAL != 1) ? (int)rank * p.b_rows : 0;
             for (int bx = lane; bx < na * nA + nb * nB; bx += 32) {
               if (bx < na * nA) {
                 const int o = bx / nA, at = bx - o * nA;
-                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : sg.map];
+                // (sg.map counts the classes of a class-group segment, not a map)
+                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : (p.grp ? 0 : sg.map)];
                 const int c1 = d.a_c1 ? sg.cls : 0;
                 const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
                 if (A_MN && p.a_merged) {
@@ -841,11 +887,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
                 // the MMA's B, or, with two B operands, all of operand r
                 const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
-                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : sg.map);
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : (p.grp ? 0 : sg.map));
                 const CUtensorMap* m = &p.mapB[mop];
-                const int c1 = d.b_c1 ? sg.cls : 0;
-                const uint32_t dst =
-                    base + na * p.a_bytes + o * p.b_bytes + (B_MN ? at * (p.b_aw * 2 * 64) : 0);
+                const int c1 = (d.b_c1 ? sg.cls : 0) + (p.grp ? at : 0);
+                const uint32_t dst = base + na * p.a_bytes + o * p.b_bytes +
+                                     (B_MN ? at * (p.b_aw * 2 * 64) : 0) + (p.grp ? at * p.box_bytes : 0);
                 if (B_MN && p.b_merged) {
                   const int x3 = (d.b_f + bsh) / p.b_aw;
                   if (PAIR) tma_load4_pair(m, dst, fb, 0, c1, kofs, x3);
@@ -921,7 +967,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
         const uint32_t acc1 = acc0 + p.n_mma;
         uint32_t accumulate = 0;
         for (int s = 0; s < d.nseg && ok; ++s) {
-          const int len = seg_at(d, s).len;
+          const Seg sgm = seg_at(d, s);
+          const int len = sgm.len;
+          // class-group mode: a one-class segment writes its class's TMEM
+          // columns with an N = grp_n MMA; the diagonal segment spans them all
+          uint32_t aoff = 0, id0 = idesc, id1 = p.idesc;
+          if (p.grp && sgm.map == 1) {
+            aoff = (uint32_t)(sgm.cls - d.roff) * (uint32_t)p.grp_n;
+            id0 = id1 = p.idesc_one;
+          }
+          const uint32_t accA = acc0 + aoff, accB = acc1 + aoff;
           for (int rem = len; rem > 0; rem -= 64) {
             if (!(mbar_try_wait(&full_bar[st], ph) || mbar_wait(&full_bar[st], ph, &s_abort))) {
               ok = false;
@@ -937,12 +992,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 if (PAIR) {
                   tc_mma_pair(acc0, a0 + ks * kA, b0 + ks * kB, idesc, accumulate);
                 } else if (single) {
-                  tc_mma(acc0, a0 + ks * kA, b0 + ks * kB, idesc, accumulate);
+                  tc_mma(accA, a0 + ks * kA, b0 + ks * kB, id0, accumulate);
                 } else {
-                  tc_mma(acc0, a0 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
-                  if (DUAL == 1) tc_mma(acc1, a0 + ks * kA, b1 + ks * kB, p.idesc, accumulate);
-                  if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, b0 + ks * kB, p.idesc, accumulate);
-                  if (DUAL == 3) tc_mma(acc0, a1 + ks * kA, b1 + ks * kB, p.idesc, 1u);
+                  tc_mma(accA, a0 + ks * kA, b0 + ks * kB, id1, accumulate);
+                  if (DUAL == 1) tc_mma(accB, a0 + ks * kA, b1 + ks * kB, id1, accumulate);
+                  if (DUAL == 2) tc_mma(accB, a1 + ks * kA, b0 + ks * kB, id1, accumulate);
+                  if (DUAL == 3) tc_mma(accA, a1 + ks * kA, b1 + ks * kB, id1, 1u);
                 }
                 accumulate = 1;
               }
@@ -953,12 +1008,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 if (PAIR) {
                   tc_mma_pair(acc0, da, db, idesc, accumulate);
                 } else if (single) {
-                  tc_mma(acc0, da, db, idesc, accumulate);
+                  tc_mma(accA, da, db, id0, accumulate);
                 } else {
-                  tc_mma(acc0, da, db, p.idesc, accumulate);
-                  if (DUAL == 1) tc_mma(acc1, da, b1 + ks * kB, p.idesc, accumulate);
-                  if (DUAL == 2) tc_mma(acc1, a1 + ks * kA, db, p.idesc, accumulate);
-                  if (DUAL == 3) tc_mma(acc0, a1 + ks * kA, b1 + ks * kB, p.idesc, 1u);
+                  tc_mma(accA, da, db, id1, accumulate);
+                  if (DUAL == 1) tc_mma(accB, da, b1 + ks * kB, id1, accumulate);
+                  if (DUAL == 2) tc_mma(accB, a1 + ks * kA, db, id1, accumulate);
+                  if (DUAL == 3) tc_mma(accA, a1 + ks * kA, b1 + ks * kB, id1, 1u);
                 }
                 accumulate = 1;
               }
@@ -1101,8 +1156,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store(&p.mapOut, sb, (int)(d.cbase + quarter * 32), d.roff,
-                        (int)(d.rbase + c0));
+              // class-group mode: TMEM columns run class by class, grp_n each
+              const int gj = p.grp ? c0 / p.grp_n : 0, gt = p.grp ? c0 - gj * p.grp_n : c0;
+              tma_store(&p.mapOut, sb, (int)(d.cbase + quarter * 32), d.roff + gj,
+                        (int)(d.rbase + gt));
               bulk_commit();
             }
           }
@@ -1650,7 +1707,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   cfg.numAttrs = 1;
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    if (!p.seg_mode) schedule_tiles(p, grid);
+    if (!p.seg_mode && !p.grp) schedule_tiles(p, grid);
     else p.use_order = 0;
     cfg.gridDim = dim3((unsigned)grid);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false>, p);
@@ -1768,6 +1825,19 @@ static bool pair_disabled() {
     v = (e && e[0] == '1') ? 0 : 1;
   }
   return v == 1;
+}
+
+// Most classes a class-group tile may hold on the swapped forward path:
+// AAL_TC_CLASS_GROUPS = 0 (one class per tile), 2 or 4 (the default); read once.
+static int grp_max() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_TC_CLASS_GROUPS");
+    v = 4;
+    if (e && (e[0] == '0' || e[0] == '1')) v = 0;
+    if (e && e[0] == '2') v = 2;
+  }
+  return v;
 }
 
 static bool position_rule_ok(const RowTypes& rt, int q, long long rows) {
@@ -1912,14 +1982,30 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     return dual ? launch<false, true, 1>(p, ntiles, s) : launch<false, true, 0>(p, ntiles, s);
   }
   const int ntok = (int)((p.Mq + 15) / 16 * 16);
+  // Class groups under Q_q: G classes share the diagonal term's weight tile
+  // and one wide MMA (G * ntok columns of TMEM per accumulator, at most 128:
+  // wider groups leave too few tiles to spread over the SMs; on the
+  // Qwen3-8B-shaped down projection G = 4 ran 50.6 us, G = 2 46.4 us, one
+  // class per tile 48.6 us)
+  int G = 0;
+  if (law == AAL_LAW_Q) {
+    for (int g = grp_max(); g >= 2; g >>= 1)
+      if (q % g == 0 && g * ntok <= 128) { G = g; break; }
+  }
   p.swap = 1;
   p.xr = ntok;
   p.wn = 128;
-  p.n_mma = ntok;
+  p.n_mma = G ? G * ntok : ntok;
   p.a_rows = 128;
-  p.b_rows = ntok;
+  p.b_rows = p.n_mma;
   p.a_aw = 64;
-  p.idesc = make_idesc(128, ntok, true, false);
+  p.idesc = make_idesc(128, p.n_mma, true, false);
+  if (G) {
+    p.grp = G;
+    p.grp_n = ntok;
+    p.idesc_one = make_idesc(128, ntok, true, false);
+    p.box_bytes = (uint32_t)ntok * 128u;
+  }
   if (!finish_plan(p, dual ? 2 : 0)) return AAL_ERR_UNSUPPORTED;
   int mg1 = 1;
   if (!map_mn(&p.mapA[0], Wg, 1, 64, 128, &p.a_merged)) return AAL_ERR_UNSUPPORTED;
@@ -1933,7 +2019,7 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
   p.n1 = 1;
   p.n2 = q;
   p.n3 = (int)(bo / 128);
-  ntiles = (long long)q * p.n2 * p.n3;
+  ntiles = (long long)(G ? q / G : q) * p.n2 * p.n3;
   return dual ? launch<true, false, 2>(p, ntiles, s) : launch<true, false, 0>(p, ntiles, s);
 }
 

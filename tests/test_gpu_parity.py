@@ -330,7 +330,8 @@ def test_square_medium(law, q, n):
 
 
 @pytest.mark.parametrize("case", ["fwd_swap", "fwd_q2xq2", "swiglu_swap", "bwd_q4", "square_b256",
-                                  "fwd_offset", "fwd_ragged_tokens"])
+                                  "fwd_offset", "fwd_ragged_tokens", "fwd_swap_groups_offset",
+                                  "swiglu_swap_48_rows", "fwd_swap_q2xq2"])
 def test_tensor_path_small_cases(case):
     T = TENSOR
     if case == "fwd_swap":
@@ -347,9 +348,41 @@ def test_tensor_path_small_cases(case):
         r = run_square("Q", 2, 512, "bf16", policy=T)
     elif case == "fwd_offset":
         r = run_project("Q", 8, 1024, 512, 1024, "bf16", seq_len=256, offset=5, policy=T)
+    elif case == "fwd_swap_groups_offset":  # 32 rows a class: groups of 4 classes, offset 5
+        r = run_project("Q", 16, 512, 1024, 2048, "bf16", seq_len=512, offset=5, policy=T)
+    elif case == "swiglu_swap_48_rows":  # 48 rows a class: gate/up in pairs of classes, down in fours
+        eh, ey, p = run_swiglu("Q", 8, 384, 1024, 2048, "bf16", seq_len=384, policy=T)
+        r = (max(eh, ey), p)
+    elif case == "fwd_swap_q2xq2":  # swapped layout without class groups (not Q_q)
+        r = run_project("Q2xQ2", 4, 256, 512, 512, "bf16", seq_len=256, policy=T)
     else:  # tokens per class not a multiple of the 128-row tile
         r = run_project("Q", 4, 4 * 200, 256, 512, "bf16", seq_len=800, policy=T)
     assert r[0] <= TOL["bf16"] and r[1] == T, r
+
+
+_ONE_CLASS_CHILD = r"""
+import sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
+from gpu_cases import TOL, run_project, run_swiglu
+import associative_algebra_block_b200 as aal
+T = aal.AAL_PATH_TENSOR
+err, p = run_project("Q", 16, 512, 1024, 2048, "bf16", seq_len=512, offset=5, policy=T)
+assert err <= TOL["bf16"] and p == T, (err, p)
+eh, ey, p = run_swiglu("Q", 8, 384, 1024, 2048, "bf16", seq_len=384, policy=T)
+assert max(eh, ey) <= TOL["bf16"] and p == T, (eh, ey, p)
+print("ok")
+"""
+
+
+def test_swapped_forward_one_class_per_tile():
+    # AAL_TC_CLASS_GROUPS=0 (read once per process) keeps one class per tile
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _ONE_CLASS_CHILD, root], capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, AAL_TC_CLASS_GROUPS="0"))
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
 
 
 # ---------------------------------------------------------------- edge cases
