@@ -36,6 +36,7 @@
 
 #include <algorithm>
 #include <queue>
+#include <atomic>
 #include <vector>
 #include <limits.h>
 #include <stdlib.h>
@@ -159,6 +160,10 @@ struct Params {
   // (idesc_one) into the class's TMEM columns.  box_bytes: one class's B box.
   int grp, grp_n;
   uint32_t idesc_one, box_bytes;
+  // Dynamic schedule (>= 0): CTA c runs tile c first, then the tiles handed
+  // out by the counter pair g_tile_ctr[dyn_slot] (next, CTAs done), so SMs
+  // that run faster take more tiles; the last CTA to finish resets the pair.
+  int dyn_slot;
   // Segment mode (forward ops with explicit or ragged row types): the rows
   // were gathered type by type into contiguous segments; tile j of the device
   // table seg_tiles (j < *seg_count) is {type, first row, end of its type's
@@ -201,6 +206,12 @@ struct TileDesc {
   int vlo, vhi;    // tile columns the epilogue writes (ragged mode)
   int split;       // >= 0: a piece of a split heavy tile (partial-sum slot), else -1
 };
+
+// Tile counters of the dynamic schedule, one pair per launch slot (launches
+// take slots round-robin, so consecutive launches, which may overlap under
+// programmatic dependent launch, never share one).  Zero between launches.
+constexpr int kDynSlots = 64;
+__device__ unsigned int g_tile_ctr[kDynSlots][2];
 
 // ------------------------------------------------------------------ PTX glue
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -1257,7 +1268,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     if (lane == 0) {
       uint32_t i = 0;
       for (int ss = tile0; ; ss += tstep, ++i) {
-        const int tile = tile_at(p, ss);
+        int tile;
+        if (p.dyn_slot >= 0) {
+          // the first tile is this CTA's own; later ones come from the counter
+          const unsigned int t =
+              i == 0 ? (unsigned)tile0 : gridDim.x + atomicAdd(&g_tile_ctr[p.dyn_slot][0], 1u);
+          tile = t < (unsigned)p.ntiles ? (int)t : -1;
+        } else {
+          tile = tile_at(p, ss);
+        }
         const uint32_t slot = i % kTileRing, ph = (i / kTileRing) & 1u;
         if (!(mbar_try_wait(&tile_empty[slot], ph ^ 1u) ||
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
@@ -1285,6 +1304,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
     else
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                    "r"(p.tmem_cols));
+  }
+  if (p.dyn_slot >= 0 && threadIdx.x == 0) {
+    // every CTA has stopped taking tiles once it gets here: the last one to
+    // arrive leaves the pair at zero for the slot's next launch
+    if (atomicAdd(&g_tile_ctr[p.dyn_slot][1], 1u) == gridDim.x - 1) {
+      atomicExch(&g_tile_ctr[p.dyn_slot][0], 0u);
+      atomicExch(&g_tile_ctr[p.dyn_slot][1], 0u);
+    }
   }
 }
 
@@ -1705,10 +1732,20 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  p.dyn_slot = -1;
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
     if (!p.seg_mode && !p.grp) schedule_tiles(p, grid);
     else p.use_order = 0;
+    // Many tiles and no cost-balanced order: hand the tiles out as CTAs free
+    // up (SMs do not all run at the same speed; on the square product the
+    // last CTA of a static stride schedule ended 25 % after the first).  The
+    // tile decoder reserves up to kTileRing tiles ahead, so with few tiles a
+    // CTA the fixed stride is as good.
+    if (!p.use_order && !p.seg_mode && ntiles >= 32LL * grid) {
+      static std::atomic<unsigned int> next_slot{0};
+      p.dyn_slot = (int)(next_slot.fetch_add(1) % kDynSlots);
+    }
     cfg.gridDim = dim3((unsigned)grid);
     const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false>, p);
     note_launch();
