@@ -60,11 +60,12 @@ ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c4-explicit", "c2-explicit", "qwe
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
     # c5: captured at n = 16384 (--config c5-n16384), x 4 for n = 32768 (4 x the tiles and bytes)
-    ("c5", "square product"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 4 * (1082815000 + 507556096), "aal_tc.cu"),
-    ("c5-n16384", "square product"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 1082815000 + 507556096, "aal_tc.cu"),
-    ("c2", "gate_up"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 23675136 + 1578240, "aal_tc.cu"),
-    ("c2", "down"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 40183808 + 1218816, "aal_tc.cu"),
-    ("c3", "gate_up"): ("bfce5740a6c8237720e0e492635094258eecbbb7841cfd143648b4e4548f2fee", 218600448 + 35601152, "aal_tc.cu"),
+    ("c5", "square product"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 4 * (1085780000 + 506635264), "aal_tc.cu"),
+    ("c5-n16384", "square product"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 1085780000 + 506635264, "aal_tc.cu"),
+    ("c2", "gate_up"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 23680512 + 1432320, "aal_tc.cu"),
+    ("c2", "down"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 40186112 + 1160960, "aal_tc.cu"),
+    ("c3", "gate_up"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 219292672 + 37301504, "aal_tc.cu"),
+    ("c3", "down"): ("6bcfa40859f1906d7e9122c680f86c057a6870075018b131ac45f5d3af58bb8f", 151107584 + 8691712, "aal_tc.cu"),
     ("c2", "decode gate_up B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 4746240, "aal_decode.cu"),
     ("c2", "decode down B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 2385152, "aal_decode.cu"),
 }
