@@ -581,9 +581,10 @@ __device__ __forceinline__ void describe_grp(const Params& p, int tile, TileDesc
   d.vhi = INT_MAX;
 }
 
+template <bool kGrp, bool kSplit>
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
   d.split = -1;
-  if (p.grp) {
+  if (kGrp && p.grp) {
     describe_grp(p, tile, d);
     return;
   }
@@ -592,7 +593,7 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     return;
   }
   int i0, i1, i2, i3, piece = 0;
-  if (p.ksplit > 1 && tile >= p.split_base) {
+  if (kSplit && p.ksplit > 1 && tile >= p.split_base) {
     // an extra piece of heavy tile dg
     const int j = tile - p.split_base, dg = j / (p.ksplit - 1);
     piece = 1 + (j - dg * (p.ksplit - 1));
@@ -662,7 +663,7 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
       const int c = i0, a = i2, t = type_of_class(p, c);
       if (p.law == AAL_LAW_Q) {
         // a in S(t, k) for Q_q: a == t (every k: one run over all groups) or k == a
-        if (a == t && p.ksplit > 1) {
+        if (kSplit && a == t && p.ksplit > 1) {
           const int k0 = piece * p.split_len;
           add_seg(d, k0, min(p.split_len, p.q * p.bo - k0), c, 0);
           d.split = ((c * p.n1 + i1) * p.n3 + i3) * p.ksplit + piece;
@@ -684,7 +685,7 @@ __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d)
     case OP_DW: {  // i0 group a, i2 group k; (i1, i3) = (row slab, column block) or swapped
       const int a = i0, k = i2;
       const int mb = p.swap ? i3 : i1, nb = p.swap ? i1 : i3;
-      if (p.law == AAL_LAW_Q && a == k && p.ksplit > 1) {
+      if (kSplit && p.law == AAL_LAW_Q && a == k && p.ksplit > 1) {
         const int k0 = piece * p.split_len;
         add_seg(d, k0, (int)min((long long)p.split_len, p.Mall - k0), 0, 1);
         d.split = ((a * p.n1 + i1) * p.n3 + i3) * p.ksplit + piece;
@@ -768,6 +769,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t smem0 = (smem_u32(dyn_smem) + 1023u) & ~1023u;
   const int S = p.stages;
+  // The optional modes exist only in the instantiations that can meet them:
+  // class groups on the swapped forward, split K on dX and dW.  The other
+  // instantiations compile without their code.
+  constexpr bool kGrp = A_MN && !B_MN && !PAIR && (DUAL == 0 || DUAL == 2);
+  constexpr bool kSplit = !PAIR && ((!A_MN && !B_MN && (DUAL == 0 || DUAL == 3)) || (A_MN && B_MN && DUAL == 0));
+  const bool grp = kGrp && p.grp;
   // Programmatic dependent launch: the next kernel of the stream may start
   // its own set-up on SMs this grid has left; it reads nothing of ours before
   // its griddepcontrol.wait, which returns once this grid has completed.
@@ -857,7 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
             if (lane == 0 && issuer) {
               // class-group mode: the segment's classes' B boxes (sg.map of them)
-              const uint32_t tx = p.grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
+              const uint32_t tx = grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
                                         : (PAIR ? 2u : 1u) * p.tx_bytes;
               mbar_expect_tx(&full_bar[st], tx);
             }
@@ -873,14 +880,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const int na = DUAL >= 2 ? 2 : 1;
             const int nb = ((DUAL == 1 && !PAIR) || DUAL == 3) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
-            const int nB = p.grp ? sg.map : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
+            const int nB = grp ? sg.map : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
             const int arow = PAIR ? (int)rank * 128 : 0;  // this CTA's half of the A tile
             const int bsh = (PAIR && DUAL != 1) ? (int)rank * p.b_rows : 0;
             for (int bx = lane; bx < na * nA + nb * nB; bx += 32) {
               if (bx < na * nA) {
                 const int o = bx / nA, at = bx - o * nA;
                 // (sg.map counts the classes of a class-group segment, not a map)
-                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : (p.grp ? 0 : sg.map)];
+                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : (grp ? 0 : sg.map)];
                 const int c1 = d.a_c1 ? sg.cls : 0;
                 const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
                 if (A_MN && p.a_merged) {
@@ -898,11 +905,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
                 // the MMA's B, or, with two B operands, all of operand r
                 const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
-                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : (p.grp ? 0 : sg.map));
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : (grp ? 0 : sg.map));
                 const CUtensorMap* m = &p.mapB[mop];
-                const int c1 = (d.b_c1 ? sg.cls : 0) + (p.grp ? at : 0);
+                const int c1 = (d.b_c1 ? sg.cls : 0) + (grp ? at : 0);
                 const uint32_t dst = base + na * p.a_bytes + o * p.b_bytes +
-                                     (B_MN ? at * (p.b_aw * 2 * 64) : 0) + (p.grp ? at * p.box_bytes : 0);
+                                     (B_MN ? at * (p.b_aw * 2 * 64) : 0) + (grp ? at * p.box_bytes : 0);
                 if (B_MN && p.b_merged) {
                   const int x3 = (d.b_f + bsh) / p.b_aw;
                   if (PAIR) tma_load4_pair(m, dst, fb, 0, c1, kofs, x3);
@@ -983,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
           // class-group mode: a one-class segment writes its class's TMEM
           // columns with an N = grp_n MMA; the diagonal segment spans them all
           uint32_t aoff = 0, id0 = idesc, id1 = p.idesc;
-          if (p.grp && sgm.map == 1) {
+          if (grp && sgm.map == 1) {
             aoff = (uint32_t)(sgm.cls - d.roff) * (uint32_t)p.grp_n;
             id0 = id1 = p.idesc_one;
           }
@@ -1099,7 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             else mbar_arrive(&tempty_bar[buf]);
           }
         }
-        if (p.ksplit > 1 && d.split >= 0) {
+        if (kSplit && p.ksplit > 1 && d.split >= 0) {
           // a piece of a split tile: its fp32 partial, TMEM lane by column
           float4* dst = reinterpret_cast<float4*>(
               p.split_ws + ((size_t)d.split * 128 + row_in_tile) * p.n_mma + c0);
@@ -1168,7 +1175,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             __syncwarp();
             if (lane == 0) {
               // class-group mode: TMEM columns run class by class, grp_n each
-              const int gj = p.grp ? c0 / p.grp_n : 0, gt = p.grp ? c0 - gj * p.grp_n : c0;
+              const int gj = grp ? c0 / p.grp_n : 0, gt = grp ? c0 - gj * p.grp_n : c0;
               tma_store(&p.mapOut, sb, (int)(d.cbase + quarter * 32), d.roff + gj,
                         (int)(d.rbase + gt));
               bulk_commit();
@@ -1282,7 +1289,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
           break;
         TileDesc d;
-        if (tile >= 0) describe(p, tile, d);
+        if (tile >= 0) describe<kGrp, kSplit>(p, tile, d);
         else d.nseg = -1;
         s_tile[slot] = d;
         mbar_arrive(&tile_full[slot]);  // release: the copy above is visible first
