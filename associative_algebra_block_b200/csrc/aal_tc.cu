@@ -160,6 +160,12 @@ struct Params {
   // (idesc_one) into the class's TMEM columns.  box_bytes: one class's B box.
   int grp, grp_n;
   uint32_t idesc_one, box_bytes;
+  // Output-group pairs (unswapped projection under Q_q, the k_tc<0,1,0,0,true>
+  // instantiation): a tile covers output groups k0 = 2 kp and k0 + 1 of one
+  // class; its first segment is X_c[., t] W(t, [k0, k0 + 2)) as one MMA of
+  // N = 2 rg_n, then X_c[., g] W(g, g) for each g != t of the pair as an MMA
+  // of N = rg_n (idesc_one) into group g's TMEM columns.
+  int rg_n;
   // Dynamic schedule (>= 0): CTA c runs tile c first, then the tiles handed
   // out by the counter pair g_tile_ctr[dyn_slot] (next, CTAs done), so SMs
   // that run faster take more tiles; the last CTA to finish resets the pair.
@@ -554,6 +560,33 @@ __device__ __forceinline__ void describe_seg(const Params& p, int tile, TileDesc
 }
 
 // tile = (pair_rank * n1 + i1) * n3 + i3; the pair is (i0, i2) of the op.
+// Segment markers of output-group-pair tiles (Seg::map): the type's own
+// segment spans both groups' columns; a diagonal segment only group j's.
+constexpr int kRgWide = 0x40, kRgNarrow = 0x20;
+
+// Output-group-pair tile (c, i1, kp): class c's 128-row block i1, output
+// groups k0 = 2 kp and k0 + 1.  Under Q_q, y_g = x_t W(t, g) + [g != t] x_g W(g, g).
+__device__ __forceinline__ void describe_rg(const Params& p, int tile, TileDesc& d) {
+  const int npair = p.q >> 1;
+  const int kp = tile % npair, r = tile / npair, i1 = r % p.n1, c = r / p.n1;
+  const int k0 = 2 * kp, t = type_of_class(p, c);
+  d.nseg = 0;
+  add_seg(d, t * p.bi, p.bi, c, kRgWide);
+  for (int j = 0; j < 2; ++j)
+    if (k0 + j != t) add_seg(d, (k0 + j) * p.bi, p.bi, c, kRgNarrow | j);
+  d.a_f = i1 * 128;
+  d.a_c1 = 1;
+  d.b_f = k0 * p.bo;
+  d.b_c1 = 0;
+  d.rbase = i1 * 128;
+  d.rstride = p.qv;
+  d.roff = c;
+  d.rlimit = p.Mq;
+  d.cbase = d.b_f;
+  d.vlo = 0;
+  d.vhi = INT_MAX;
+}
+
 // Class-group tile (cg, k, i3): classes c0 = cg * grp ... c0 + grp - 1, output
 // group k, 128-column block i3 of it.  Under Q_q every class's rows add
 // X_c[., k] W(k, k) (the diagonal term, one segment over all grp classes: B
@@ -581,9 +614,13 @@ __device__ __forceinline__ void describe_grp(const Params& p, int tile, TileDesc
   d.vhi = INT_MAX;
 }
 
-template <bool kGrp, bool kSplit>
+template <bool kGrp, bool kSplit, bool kRg>
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
   d.split = -1;
+  if (kRg) {
+    describe_rg(p, tile, d);
+    return;
+  }
   if (kGrp && p.grp) {
     describe_grp(p, tile, d);
     return;
@@ -750,7 +787,7 @@ __device__ __forceinline__ bool take_tile(const TileDesc* ring, uint64_t* full, 
 // each CTA loads its half of A's rows and of B's columns (for DUAL == 1, CTA r
 // loads B operand r), only the pair's first CTA issues MMAs and counts the
 // transaction bytes, and each CTA drains its own 128 TMEM lanes.
-template <bool A_MN, bool B_MN, int DUAL, bool PAIR>
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR, bool RG = false>
 __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Params p) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[kMaxStages];
@@ -774,6 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   // instantiations compile without their code.
   constexpr bool kGrp = A_MN && !B_MN && !PAIR && (DUAL == 0 || DUAL == 2);
   constexpr bool kSplit = !PAIR && ((!A_MN && !B_MN && (DUAL == 0 || DUAL == 3)) || (A_MN && B_MN && DUAL == 0));
+  constexpr bool kRg = RG && !A_MN && B_MN && DUAL == 0 && !PAIR;  // output-group pairs
   const bool grp = kGrp && p.grp;
   // Programmatic dependent launch: the next kernel of the stream may start
   // its own set-up on SMs this grid has left; it reads nothing of ours before
@@ -864,8 +902,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const uint32_t fb = PAIR ? mapa_rank(smem_u32(&full_bar[st]), 0) : smem_u32(&full_bar[st]);
             if (lane == 0 && issuer) {
               // class-group mode: the segment's classes' B boxes (sg.map of them)
-              const uint32_t tx = grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
-                                        : (PAIR ? 2u : 1u) * p.tx_bytes;
+              const uint32_t tx =
+                  grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
+                      : kRg ? p.a_bytes + (uint32_t)(sg.map == kRgWide ? 2 : 1) * (uint32_t)p.rg_n * 128u
+                            : (PAIR ? 2u : 1u) * p.tx_bytes;
               mbar_expect_tx(&full_bar[st], tx);
             }
             if (lane == 0) atomicMax(&s_last_chunk[st], (int)it);
@@ -880,14 +920,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             const int na = DUAL >= 2 ? 2 : 1;
             const int nb = ((DUAL == 1 && !PAIR) || DUAL == 3) ? 2 : 1;
             const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
-            const int nB = grp ? sg.map : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
+            const int nB = grp ? sg.map
+                           : kRg ? (sg.map == kRgWide ? 2 * p.rg_n : p.rg_n) / p.b_aw
+                                 : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
             const int arow = PAIR ? (int)rank * 128 : 0;  // this CTA's half of the A tile
             const int bsh = (PAIR && DUAL != 1) ? (int)rank * p.b_rows : 0;
             for (int bx = lane; bx < na * nA + nb * nB; bx += 32) {
               if (bx < na * nA) {
                 const int o = bx / nA, at = bx - o * nA;
                 // (sg.map counts the classes of a class-group segment, not a map)
-                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : (grp ? 0 : sg.map)];
+                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : ((grp || kRg) ? 0 : sg.map)];
                 const int c1 = d.a_c1 ? sg.cls : 0;
                 const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
                 if (A_MN && p.a_merged) {
@@ -905,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
                 // the MMA's B, or, with two B operands, all of operand r
                 const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
-                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : (grp ? 0 : sg.map));
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : ((grp || kRg) ? 0 : sg.map));
                 const CUtensorMap* m = &p.mapB[mop];
                 const int c1 = (d.b_c1 ? sg.cls : 0) + (grp ? at : 0);
                 const uint32_t dst = base + na * p.a_bytes + o * p.b_bytes +
@@ -915,7 +957,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                   if (PAIR) tma_load4_pair(m, dst, fb, 0, c1, kofs, x3);
                   else tma_load4(m, dst, &full_bar[st], 0, c1, kofs, x3);
                 } else {
-                  const int x0 = B_MN ? d.b_f + bsh + at * p.b_aw : kofs;
+                  // output-group pairs: a diagonal segment's columns are group j's
+                  const int rgo = (kRg && sg.map != kRgWide) ? (sg.map & 1) * p.rg_n : 0;
+                  const int x0 = B_MN ? d.b_f + bsh + at * p.b_aw + rgo : kofs;
                   const int x2 = B_MN ? kofs : d.b_f + bsh;
                   if (PAIR) tma_load_pair(m, dst, fb, x0, c1, x2);
                   else tma_load(m, dst, &full_bar[st], x0, c1, x2);
@@ -992,6 +1036,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
           uint32_t aoff = 0, id0 = idesc, id1 = p.idesc;
           if (grp && sgm.map == 1) {
             aoff = (uint32_t)(sgm.cls - d.roff) * (uint32_t)p.grp_n;
+            id0 = id1 = p.idesc_one;
+          }
+          if (kRg && sgm.map != kRgWide) {
+            aoff = (uint32_t)(sgm.map & 1) * (uint32_t)p.rg_n;
             id0 = id1 = p.idesc_one;
           }
           const uint32_t accA = acc0 + aoff, accB = acc1 + aoff;
@@ -1289,7 +1337,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
           break;
         TileDesc d;
-        if (tile >= 0) describe<kGrp, kSplit>(p, tile, d);
+        if (tile >= 0) describe<kGrp, kSplit, kRg>(p, tile, d);
         else d.nseg = -1;
         s_tile[slot] = d;
         mbar_arrive(&tile_full[slot]);  // release: the copy above is visible first
@@ -1696,7 +1744,7 @@ static int test_stall_enabled() {
   return (e && e[0] == '1') ? 1 : 0;
 }
 
-template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false>
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false, bool RG = false>
 static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (ntiles <= 0) return AAL_OK;
   if (ntiles > INT_MAX) return AAL_ERR_UNSUPPORTED;
@@ -1721,7 +1769,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return AAL_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    if (cudaFuncSetAttribute(k_tc<A_MN, B_MN, DUAL, PAIR>,
+    if (cudaFuncSetAttribute(k_tc<A_MN, B_MN, DUAL, PAIR, RG>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBudget + 1024) != cudaSuccess)
       return AAL_ERR_CUDA;
@@ -1742,7 +1790,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   p.dyn_slot = -1;
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    if (!p.seg_mode && !p.grp) schedule_tiles(p, grid);
+    if (!p.seg_mode && !p.grp && !RG) schedule_tiles(p, grid);
     else p.use_order = 0;
     // Many tiles and no cost-balanced order: hand the tiles out as CTAs free
     // up (SMs do not all run at the same speed; on the square product the
@@ -1754,7 +1802,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
       p.dyn_slot = (int)(next_slot.fetch_add(1) % kDynSlots);
     }
     cfg.gridDim = dim3((unsigned)grid);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false>, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false, RG>, p);
     note_launch();
     return cuda_status(e);
   }
@@ -1884,6 +1932,17 @@ static int grp_max() {
   return v;
 }
 
+// AAL_TC_GROUP_PAIRS=0 keeps one output group per tile on the unswapped
+// projection (read once).
+static bool rg_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_TC_GROUP_PAIRS");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 static bool position_rule_ok(const RowTypes& rt, int q, long long rows) {
   return rt.kind == kTypesPosition && rt.seq_len % q == 0 && rows % q == 0 && rows > 0;
 }
@@ -1994,6 +2053,32 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     p.n3 = (int)(bo / n);
     ntiles = (long long)q * p.n1 * p.n2 * p.n3;
     return dual ? launch<false, true, 1, true>(p, ntiles, s) : launch<false, true, 0, true>(p, ntiles, s);
+  }
+  if (!swap && !dual && law == AAL_LAW_Q && q % 2 == 0 && 2 * bo <= 256 && rg_enabled()) {
+    // Output-group pairs: the type's own segment x_t W(t, [k0, k0 + 2)) as
+    // one MMA over both groups' columns, the two diagonal terms into their
+    // column ranges (half the tiles of one group each, and fewer MMAs)
+    const int n = (int)(2 * bo);
+    p.swap = 0;
+    p.xr = 128;
+    p.wn = n;
+    p.n_mma = n;
+    p.a_rows = 128;
+    p.b_rows = n;
+    p.b_aw = bo % 64 == 0 ? 64 : 16;
+    p.rg_n = (int)bo;
+    p.idesc = make_idesc(128, n, false, true);
+    p.idesc_one = make_idesc(128, (int)bo, false, true);
+    if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], X, q, 128)) return AAL_ERR_UNSUPPORTED;
+    if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    p.b_merged = 0;  // a diagonal segment loads only its group's atoms
+    if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = (int)((p.Mq + 127) / 128);
+    p.n2 = q;
+    p.n3 = 1;
+    ntiles = (long long)q * p.n1 * (q / 2);
+    return launch<false, true, 0, false, true>(p, ntiles, s);
   }
   if (!swap) {
     const int n = pick_n(bo, dual ? 128 : 256);

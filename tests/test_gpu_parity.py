@@ -331,7 +331,8 @@ def test_square_medium(law, q, n):
 
 @pytest.mark.parametrize("case", ["fwd_swap", "fwd_q2xq2", "swiglu_swap", "bwd_q4", "square_b256",
                                   "fwd_offset", "fwd_ragged_tokens", "fwd_swap_groups_offset",
-                                  "swiglu_swap_48_rows", "fwd_swap_q2xq2"])
+                                  "swiglu_swap_48_rows", "fwd_swap_q2xq2", "fwd_group_pairs_q2",
+                                  "fwd_group_pairs_48"])
 def test_tensor_path_small_cases(case):
     T = TENSOR
     if case == "fwd_swap":
@@ -355,6 +356,10 @@ def test_tensor_path_small_cases(case):
         r = (max(eh, ey), p)
     elif case == "fwd_swap_q2xq2":  # swapped layout without class groups (not Q_q)
         r = run_project("Q2xQ2", 4, 256, 512, 512, "bf16", seq_len=256, policy=T)
+    elif case == "fwd_group_pairs_q2":  # one pair of output groups, 200 rows a class
+        r = run_project("Q", 2, 400, 256, 128, "bf16", seq_len=400, policy=T)
+    elif case == "fwd_group_pairs_48":  # 48-column groups in pairs, offset 3, a partial row block
+        r = run_project("Q", 16, 16 * 160, 2048, 768, "bf16", seq_len=16 * 160, offset=3, policy=T)
     else:  # tokens per class not a multiple of the 128-row tile
         r = run_project("Q", 4, 4 * 200, 256, 512, "bf16", seq_len=800, policy=T)
     assert r[0] <= TOL["bf16"] and r[1] == T, r
@@ -372,6 +377,30 @@ eh, ey, p = run_swiglu("Q", 8, 384, 1024, 2048, "bf16", seq_len=384, policy=T)
 assert max(eh, ey) <= TOL["bf16"] and p == T, (eh, ey, p)
 print("ok")
 """
+
+
+_ONE_GROUP_CHILD = r"""
+import sys
+sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
+from gpu_cases import TOL, run_project
+import associative_algebra_block_b200 as aal
+T = aal.AAL_PATH_TENSOR
+for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512, 1024, 256, 5)):
+    err, p = run_project("Q", q, M, din, dout, "bf16", seq_len=seq, offset=off, policy=T)
+    assert err <= TOL["bf16"] and p == T, (q, err, p)
+print("ok")
+"""
+
+
+def test_unswapped_projection_one_output_group_per_tile():
+    # AAL_TC_GROUP_PAIRS=0 (read once per process) keeps one output group per tile
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _ONE_GROUP_CHILD, root], capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, AAL_TC_GROUP_PAIRS="0"))
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
 
 
 def test_swapped_forward_one_class_per_tile():
