@@ -382,6 +382,26 @@ AAL_API int64_t aal_launch_count(int32_t reset);
 /* Library version as major*10000 + minor*100 + patch. */
 AAL_API int32_t aal_version(void);
 
+/*
+ * Environment switches (read once per process, except AAL_TEST_STALL).  The
+ * defaults are the measured-fastest choices; the alternatives compute the
+ * same products and stay available for comparison and testing.
+ *   AAL_TC_PAIR=1            CTA pairs (tcgen05 cta_group::2, M = 256) for the
+ *                            unswapped forward (default off: measured slower).
+ *   AAL_TC_CLASS_GROUPS=0|2|4  most row types a tile of the swapped forward
+ *                            holds (default 4; wider than 128 columns is never
+ *                            chosen); 0 keeps one type per tile.
+ *   AAL_TC_GROUP_PAIRS=0     one output group per tile on the unswapped Q_q
+ *                            projection (default: pairs of groups).
+ *   AAL_DECODE_MMA=0         SIMT decode kernels instead of the tensor-core one.
+ *   AAL_DECODE_TYPED=0       the cluster decode kernel for single-type batches.
+ *   AAL_FFN_DECODE_FUSED=1   the one-launch FFN decode (default off: slower).
+ *   AAL_TEST_STALL=1         test hook: the tcgen05 kernel's MMA thread waits on
+ *                            a barrier nothing arrives on until the bounded
+ *                            wait runs out (AAL_ERR_DEVICE_TIMEOUT); read at
+ *                            every launch.
+ */
+
 #ifdef __cplusplus
 }
 #endif
