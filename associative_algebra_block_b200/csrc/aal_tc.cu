@@ -566,22 +566,26 @@ constexpr int kRgWide = 0x40, kRgNarrow = 0x20;
 
 // Output-group-pair tile (c, i1, kp): class c's 128-row block i1, output
 // groups k0 = 2 kp and k0 + 1.  Under Q_q, y_g = x_t W(t, g) + [g != t] x_g W(g, g).
+// For the square product the class is row block i (Z_ig = X_ii W_ig + [g != i]
+// X_ig W_gg) and its rows are plain rows of X and Z.
 __device__ __forceinline__ void describe_rg(const Params& p, int tile, TileDesc& d) {
   const int npair = p.q >> 1;
   const int kp = tile % npair, r = tile / npair, i1 = r % p.n1, c = r / p.n1;
-  const int k0 = 2 * kp, t = type_of_class(p, c);
+  const bool sq = p.op == OP_SQUARE;
+  const int k0 = 2 * kp, t = sq ? c : type_of_class(p, c);
+  const int cls = sq ? 0 : c;
   d.nseg = 0;
-  add_seg(d, t * p.bi, p.bi, c, kRgWide);
+  add_seg(d, t * p.bi, p.bi, cls, kRgWide);
   for (int j = 0; j < 2; ++j)
-    if (k0 + j != t) add_seg(d, (k0 + j) * p.bi, p.bi, c, kRgNarrow | j);
-  d.a_f = i1 * 128;
-  d.a_c1 = 1;
+    if (k0 + j != t) add_seg(d, (k0 + j) * p.bi, p.bi, cls, kRgNarrow | j);
+  d.a_f = sq ? c * p.bi + i1 * 128 : i1 * 128;
+  d.a_c1 = sq ? 0 : 1;
   d.b_f = k0 * p.bo;
   d.b_c1 = 0;
-  d.rbase = i1 * 128;
-  d.rstride = p.qv;
-  d.roff = c;
-  d.rlimit = p.Mq;
+  d.rbase = d.a_f;
+  d.rstride = sq ? 1 : p.qv;
+  d.roff = sq ? 0 : c;
+  d.rlimit = sq ? LLONG_MAX : p.Mq;
   d.cbase = d.b_f;
   d.vlo = 0;
   d.vhi = INT_MAX;
@@ -2408,6 +2412,28 @@ aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const a
   p.bo = (int)b;
   p.out = (__nv_bfloat16*)Z.ptr;
   p.ldo = Z.ld;
+  if (law == AAL_LAW_Q && q % 2 == 0 && b == 128 && rg_enabled()) {
+    // column-block pairs: X_ii W_i,[k0, k0 + 2) as one N = 256 MMA, then the
+    // diagonal terms X_ig W_gg into their blocks' column ranges
+    p.xr = 128;
+    p.wn = 256;
+    p.n_mma = 256;
+    p.a_rows = 128;
+    p.b_rows = 256;
+    p.b_aw = 64;
+    p.rg_n = 128;
+    p.idesc = make_idesc(128, 256, false, true);
+    p.idesc_one = make_idesc(128, 128, false, true);
+    if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], X, 1, 128)) return AAL_ERR_UNSUPPORTED;
+    if (!map_mnmajor(&p.mapB[0], W, 1, 64)) return AAL_ERR_UNSUPPORTED;
+    p.b_merged = 0;
+    if (!out_map(p, Z, 1)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = 1;
+    p.n2 = q;
+    p.n3 = 1;
+    return launch<false, true, 0, false, true>(p, (long long)(q / 2) * q, s);
+  }
   const int nn = pick_n(b, 256);
   p.xr = 128;
   p.wn = nn;

@@ -322,7 +322,8 @@ def test_c5_square_full_size_sampled_tiles():
     assert worst <= TOL["bf16"], worst
 
 
-@pytest.mark.parametrize("law,q,n", [("Q", 4, 512), ("Q", 16, 2048), ("Q2xQ2", 4, 256)])
+# Q_q with 128-wide blocks and even q runs column-block pairs; odd q one block a tile
+@pytest.mark.parametrize("law,q,n", [("Q", 4, 512), ("Q", 16, 2048), ("Q2xQ2", 4, 256), ("Q", 3, 384)])
 def test_square_medium(law, q, n):
     err, path = run_square(law, q, n, "bf16")
     assert err <= TOL["bf16"], err
@@ -382,12 +383,14 @@ print("ok")
 _ONE_GROUP_CHILD = r"""
 import sys
 sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
-from gpu_cases import TOL, run_project
+from gpu_cases import TOL, run_project, run_square
 import associative_algebra_block_b200 as aal
 T = aal.AAL_PATH_TENSOR
 for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512, 1024, 256, 5)):
     err, p = run_project("Q", q, M, din, dout, "bf16", seq_len=seq, offset=off, policy=T)
     assert err <= TOL["bf16"] and p == T, (q, err, p)
+err, p = run_square("Q", 4, 512, "bf16", policy=T)
+assert err <= TOL["bf16"] and p == T, (err, p)
 print("ok")
 """
 
