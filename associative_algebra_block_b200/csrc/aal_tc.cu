@@ -591,6 +591,33 @@ __device__ __forceinline__ void describe_rg(const Params& p, int tile, TileDesc&
   d.vhi = INT_MAX;
 }
 
+// Class-pair tile (cp, k, i3) of the unswapped projection (at most 64 rows a
+// type): the 128 A rows are classes c0 = 2 cp and c0 + 1, 64 rows each.  The
+// diagonal term X_c[., k] W(k, k) is one MMA over both; X_c[., t] W(t, k)
+// (t = type of c != k) loads class c's rows and zeros in the other half.
+constexpr int kCpBoth = 0x50, kCpOne = 0x60;
+__device__ __forceinline__ void describe_cp(const Params& p, int tile, TileDesc& d) {
+  const int i3 = tile % p.n3, r = tile / p.n3, k = r % p.q, cp = r / p.q;
+  const int c0 = 2 * cp;
+  d.nseg = 0;
+  add_seg(d, k * p.bi, p.bi, c0, kCpBoth);
+  for (int j = 0; j < 2; ++j) {
+    const int t = type_of_class(p, c0 + j);
+    if (t != k) add_seg(d, t * p.bi, p.bi, c0 + j, kCpOne | j);
+  }
+  d.a_f = 0;
+  d.a_c1 = 1;
+  d.b_f = k * p.bo + i3 * p.wn;
+  d.b_c1 = 0;
+  d.rbase = 0;
+  d.rstride = p.qv;
+  d.roff = c0;
+  d.rlimit = p.Mq;
+  d.cbase = d.b_f;
+  d.vlo = 0;
+  d.vhi = INT_MAX;
+}
+
 // Class-group tile (cg, k, i3): classes c0 = cg * grp ... c0 + grp - 1, output
 // group k, 128-column block i3 of it.  Under Q_q every class's rows add
 // X_c[., k] W(k, k) (the diagonal term, one segment over all grp classes: B
@@ -618,11 +645,15 @@ __device__ __forceinline__ void describe_grp(const Params& p, int tile, TileDesc
   d.vhi = INT_MAX;
 }
 
-template <bool kGrp, bool kSplit, bool kRg>
+template <bool kGrp, bool kSplit, bool kRg, bool kCp>
 __device__ __forceinline__ void describe(const Params& p, int tile, TileDesc& d) {
   d.split = -1;
   if (kRg) {
     describe_rg(p, tile, d);
+    return;
+  }
+  if (kCp) {
+    describe_cp(p, tile, d);
     return;
   }
   if (kGrp && p.grp) {
@@ -791,7 +822,8 @@ __device__ __forceinline__ bool take_tile(const TileDesc* ring, uint64_t* full, 
 // each CTA loads its half of A's rows and of B's columns (for DUAL == 1, CTA r
 // loads B operand r), only the pair's first CTA issues MMAs and counts the
 // transaction bytes, and each CTA drains its own 128 TMEM lanes.
-template <bool A_MN, bool B_MN, int DUAL, bool PAIR, bool RG = false>
+// MODE: 0 plain; 1 output-group pairs; 2 class pairs (unswapped projection)
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR, int MODE = 0>
 __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Params p) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ __align__(8) uint64_t full_bar[kMaxStages];
@@ -815,7 +847,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   // instantiations compile without their code.
   constexpr bool kGrp = A_MN && !B_MN && !PAIR && (DUAL == 0 || DUAL == 2);
   constexpr bool kSplit = !PAIR && ((!A_MN && !B_MN && (DUAL == 0 || DUAL == 3)) || (A_MN && B_MN && DUAL == 0));
-  constexpr bool kRg = RG && !A_MN && B_MN && DUAL == 0 && !PAIR;  // output-group pairs
+  constexpr bool kRg = MODE == 1 && !A_MN && B_MN && DUAL == 0 && !PAIR;  // output-group pairs
+  constexpr bool kCp = MODE == 2 && !A_MN && B_MN && DUAL == 0 && !PAIR;  // class pairs
   const bool grp = kGrp && p.grp;
   // Programmatic dependent launch: the next kernel of the stream may start
   // its own set-up on SMs this grid has left; it reads nothing of ours before
@@ -923,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             } else {
             const int na = DUAL >= 2 ? 2 : 1;
             const int nb = ((DUAL == 1 && !PAIR) || DUAL == 3) ? 2 : 1;
-            const int nA = (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
+            const int nA = kCp ? 2 : (A_MN && !p.a_merged) ? p.a_rows / p.a_aw : 1;  // boxes per A operand
             const int nB = grp ? sg.map
                            : kRg ? (sg.map == kRgWide ? 2 * p.rg_n : p.rg_n) / p.b_aw
                                  : ((B_MN && !p.b_merged) ? p.b_rows / p.b_aw : 1);  // boxes per B operand
@@ -933,9 +966,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               if (bx < na * nA) {
                 const int o = bx / nA, at = bx - o * nA;
                 // (sg.map counts the classes of a class-group segment, not a map)
-                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : ((grp || kRg) ? 0 : sg.map)];
-                const int c1 = d.a_c1 ? sg.cls : 0;
-                const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0);
+                const CUtensorMap* m = &p.mapA[DUAL >= 2 ? o : ((grp || kRg || kCp) ? 0 : sg.map)];
+                // class pairs: box at = class c0 + at's 64 rows; a one-class segment
+                // reads rows past the end (zeros) for the other class
+                const bool cp_zero = kCp && sg.map != kCpBoth && at != (sg.map & 1);
+                const int c1 = kCp ? d.roff + at : (d.a_c1 ? sg.cls : 0);
+                const uint32_t dst = base + o * p.a_bytes + (A_MN ? at * (p.a_aw * 2 * 64) : 0) +
+                                     (kCp ? at * 64 * 128 : 0);
                 if (A_MN && p.a_merged) {
                   // all atoms at once: coordinates (col in atom, class, K row, atom)
                   const int x3 = (d.a_f + arow) / p.a_aw;
@@ -943,7 +980,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                   else tma_load4(m, dst, &full_bar[st], 0, c1, kofs, x3);
                 } else {
                   const int x0 = A_MN ? d.a_f + arow + at * p.a_aw : kofs;
-                  const int x2 = A_MN ? kofs : d.a_f + arow;
+                  const int x2 = A_MN ? kofs : (cp_zero ? 64 : d.a_f + arow);
                   if (PAIR) tma_load_pair(m, dst, fb, x0, c1, x2);
                   else tma_load(m, dst, &full_bar[st], x0, c1, x2);
                 }
@@ -951,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
                 // B: for a pair, CTA r holds columns [r*b_rows, (r+1)*b_rows) of
                 // the MMA's B, or, with two B operands, all of operand r
                 const int jb = bx - na * nA, o = jb / nB, at = jb - o * nB;
-                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : ((grp || kRg) ? 0 : sg.map));
+                const int mop = DUAL == 1 ? (PAIR ? (int)rank : o) : (DUAL == 3 ? o : ((grp || kRg || kCp) ? 0 : sg.map));
                 const CUtensorMap* m = &p.mapB[mop];
                 const int c1 = (d.b_c1 ? sg.cls : 0) + (grp ? at : 0);
                 const uint32_t dst = base + na * p.a_bytes + o * p.b_bytes +
@@ -1211,8 +1248,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
             fence_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store(&p.mapOut, sb, (int)(d.cbase + c0), d.roff,
-                        (int)(d.rbase + quarter * 32));
+              // class pairs: TMEM lanes 0-63 are class roff's rows, 64-127 the next class's
+              if (kCp)
+                tma_store(&p.mapOut, sb, (int)(d.cbase + c0), d.roff + (quarter >> 1),
+                          (int)(d.rbase + (quarter & 1) * 32));
+              else
+                tma_store(&p.mapOut, sb, (int)(d.cbase + c0), d.roff,
+                          (int)(d.rbase + quarter * 32));
               bulk_commit();
             }
           } else {
@@ -1341,7 +1383,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               mbar_wait(&tile_empty[slot], ph ^ 1u, &s_abort)))
           break;
         TileDesc d;
-        if (tile >= 0) describe<kGrp, kSplit, kRg>(p, tile, d);
+        if (tile >= 0) describe<kGrp, kSplit, kRg, kCp>(p, tile, d);
         else d.nseg = -1;
         s_tile[slot] = d;
         mbar_arrive(&tile_full[slot]);  // release: the copy above is visible first
@@ -1748,7 +1790,7 @@ static int test_stall_enabled() {
   return (e && e[0] == '1') ? 1 : 0;
 }
 
-template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false, bool RG = false>
+template <bool A_MN, bool B_MN, int DUAL, bool PAIR = false, int MODE = 0>
 static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (ntiles <= 0) return AAL_OK;
   if (ntiles > INT_MAX) return AAL_ERR_UNSUPPORTED;
@@ -1773,7 +1815,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return AAL_ERR_CUDA;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    if (cudaFuncSetAttribute(k_tc<A_MN, B_MN, DUAL, PAIR, RG>,
+    if (cudaFuncSetAttribute(k_tc<A_MN, B_MN, DUAL, PAIR, MODE>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSmemBudget + 1024) != cudaSuccess)
       return AAL_ERR_CUDA;
@@ -1794,7 +1836,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
   p.dyn_slot = -1;
   if (!PAIR) {
     const int grid = (int)(ntiles < sms ? ntiles : sms);
-    if (!p.seg_mode && !p.grp && !RG) schedule_tiles(p, grid);
+    if (!p.seg_mode && !p.grp && MODE == 0) schedule_tiles(p, grid);
     else p.use_order = 0;
     // Many tiles and no cost-balanced order: hand the tiles out as CTAs free
     // up (SMs do not all run at the same speed; on the square product the
@@ -1806,7 +1848,7 @@ static aal_status launch(Params& p, long long ntiles, cudaStream_t s) {
       p.dyn_slot = (int)(next_slot.fetch_add(1) % kDynSlots);
     }
     cfg.gridDim = dim3((unsigned)grid);
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false, RG>, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_tc<A_MN, B_MN, DUAL, false, MODE>, p);
     note_launch();
     return cuda_status(e);
   }
@@ -1936,6 +1978,17 @@ static int grp_max() {
   return v;
 }
 
+// AAL_TC_CLASS_PAIRS=0 keeps one row type per tile on the unswapped
+// projection when a type has at most 64 rows (read once).
+static bool cp_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("AAL_TC_CLASS_PAIRS");
+    v = (e && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
 // AAL_TC_GROUP_PAIRS=0 keeps one output group per tile on the unswapped
 // projection (read once).
 static bool rg_enabled() {
@@ -2058,6 +2111,29 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     ntiles = (long long)q * p.n1 * p.n2 * p.n3;
     return dual ? launch<false, true, 1, true>(p, ntiles, s) : launch<false, true, 0, true>(p, ntiles, s);
   }
+  if (!swap && !dual && law == AAL_LAW_Q && q % 2 == 0 && p.Mq <= 64 && cp_enabled()) {
+    // Class pairs: at most 64 rows a type fill half of a 128-row tile; two
+    // types share the tile, the diagonal term as one MMA over both
+    const int n = pick_n(bo, 256);
+    if (!n) return AAL_ERR_UNSUPPORTED;
+    p.swap = 0;
+    p.xr = 128;
+    p.wn = n;
+    p.n_mma = n;
+    p.a_rows = 128;
+    p.b_rows = n;
+    p.b_aw = n % 64 == 0 ? 64 : 16;
+    p.idesc = make_idesc(128, n, false, true);
+    if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], X, q, 64)) return AAL_ERR_UNSUPPORTED;
+    if (!map_mn(&p.mapB[0], Wg, 1, p.b_aw, p.b_rows, &p.b_merged)) return AAL_ERR_UNSUPPORTED;
+    if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = 1;
+    p.n2 = q;
+    p.n3 = (int)(bo / n);
+    ntiles = (long long)(q / 2) * q * p.n3;
+    return launch<false, true, 0, false, 2>(p, ntiles, s);
+  }
   if (!swap && !dual && law == AAL_LAW_Q && q % 2 == 0 && 2 * bo <= 256 && rg_enabled()) {
     // Output-group pairs: the type's own segment x_t W(t, [k0, k0 + 2)) as
     // one MMA over both groups' columns, the two diagonal terms into their
@@ -2082,7 +2158,7 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     p.n2 = q;
     p.n3 = 1;
     ntiles = (long long)q * p.n1 * (q / 2);
-    return launch<false, true, 0, false, true>(p, ntiles, s);
+    return launch<false, true, 0, false, 1>(p, ntiles, s);
   }
   if (!swap) {
     const int n = pick_n(bo, dual ? 128 : 256);
@@ -2432,7 +2508,7 @@ aal_status tc_square(int law, int q, const aal_mat& X, const aal_mat& W, const a
     p.n1 = 1;
     p.n2 = q;
     p.n3 = 1;
-    return launch<false, true, 0, false, true>(p, (long long)(q / 2) * q, s);
+    return launch<false, true, 0, false, 1>(p, (long long)(q / 2) * q, s);
   }
   const int nn = pick_n(b, 256);
   p.xr = 128;

@@ -392,7 +392,10 @@ AAL_API int32_t aal_version(void);
  *                            holds (default 4; wider than 128 columns is never
  *                            chosen); 0 keeps one type per tile.
  *   AAL_TC_GROUP_PAIRS=0     one output group per tile on the unswapped Q_q
- *                            projection (default: pairs of groups).
+ *                            projection and square product (default: pairs).
+ *   AAL_TC_CLASS_PAIRS=0     one row type per tile on the unswapped Q_q
+ *                            projection when a type has at most 64 rows
+ *                            (default: two types share a tile).
  *   AAL_DECODE_MMA=0         SIMT decode kernels instead of the tensor-core one.
  *   AAL_DECODE_TYPED=0       the cluster decode kernel for single-type batches.
  *   AAL_FFN_DECODE_FUSED=1   the one-launch FFN decode (default off: slower).

@@ -333,7 +333,8 @@ def test_square_medium(law, q, n):
 @pytest.mark.parametrize("case", ["fwd_swap", "fwd_q2xq2", "swiglu_swap", "bwd_q4", "square_b256",
                                   "fwd_offset", "fwd_ragged_tokens", "fwd_swap_groups_offset",
                                   "swiglu_swap_48_rows", "fwd_swap_q2xq2", "fwd_group_pairs_q2",
-                                  "fwd_group_pairs_48"])
+                                  "fwd_group_pairs_48", "fwd_class_pairs_48_rows",
+                                  "fwd_class_pairs_q4"])
 def test_tensor_path_small_cases(case):
     T = TENSOR
     if case == "fwd_swap":
@@ -361,6 +362,10 @@ def test_tensor_path_small_cases(case):
         r = run_project("Q", 2, 400, 256, 128, "bf16", seq_len=400, policy=T)
     elif case == "fwd_group_pairs_48":  # 48-column groups in pairs, offset 3, a partial row block
         r = run_project("Q", 16, 16 * 160, 2048, 768, "bf16", seq_len=16 * 160, offset=3, policy=T)
+    elif case == "fwd_class_pairs_48_rows":  # 48 rows a type: two types share a tile, offset 3
+        r = run_project("Q", 16, 16 * 48, 512, 16 * 80, "bf16", seq_len=16 * 48, offset=3, policy=T)
+    elif case == "fwd_class_pairs_q4":  # 64 rows a type, 96-column groups
+        r = run_project("Q", 4, 256, 256, 384, "bf16", seq_len=256, policy=T)
     else:  # tokens per class not a multiple of the 128-row tile
         r = run_project("Q", 4, 4 * 200, 256, 512, "bf16", seq_len=800, policy=T)
     assert r[0] <= TOL["bf16"] and r[1] == T, r
@@ -386,7 +391,8 @@ sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
 from gpu_cases import TOL, run_project, run_square
 import associative_algebra_block_b200 as aal
 T = aal.AAL_PATH_TENSOR
-for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512, 1024, 256, 5)):
+for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512, 1024, 256, 5),
+                                   (16, 768, 512, 1280, 768, 3)):
     err, p = run_project("Q", q, M, din, dout, "bf16", seq_len=seq, offset=off, policy=T)
     assert err <= TOL["bf16"] and p == T, (q, err, p)
 err, p = run_square("Q", 4, 512, "bf16", policy=T)
@@ -396,13 +402,14 @@ print("ok")
 
 
 def test_unswapped_projection_one_output_group_per_tile():
-    # AAL_TC_GROUP_PAIRS=0 (read once per process) keeps one output group per tile
+    # AAL_TC_GROUP_PAIRS=0 and AAL_TC_CLASS_PAIRS=0 (read once per process) keep one
+    # output group and one row type per tile
     import os
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, "-c", _ONE_GROUP_CHILD, root], capture_output=True, text=True,
-                       timeout=600, env=dict(os.environ, AAL_TC_GROUP_PAIRS="0"))
+                       timeout=600, env=dict(os.environ, AAL_TC_GROUP_PAIRS="0", AAL_TC_CLASS_PAIRS="0"))
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
 
 
