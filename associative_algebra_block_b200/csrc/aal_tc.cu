@@ -847,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
   // instantiations compile without their code.
   constexpr bool kGrp = A_MN && !B_MN && !PAIR && (DUAL == 0 || DUAL == 2);
   constexpr bool kSplit = !PAIR && ((!A_MN && !B_MN && (DUAL == 0 || DUAL == 3)) || (A_MN && B_MN && DUAL == 0));
-  constexpr bool kRg = MODE == 1 && !A_MN && B_MN && DUAL == 0 && !PAIR;  // output-group pairs
+  constexpr bool kRg = MODE == 1 && !A_MN && B_MN && (DUAL == 0 || DUAL == 1) && !PAIR;  // output-group pairs
   constexpr bool kCp = MODE == 2 && !A_MN && B_MN && DUAL == 0 && !PAIR;  // class pairs
   const bool grp = kGrp && p.grp;
   // Programmatic dependent launch: the next kernel of the stream may start
@@ -941,7 +941,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_tc(const __grid_constant__ Para
               // class-group mode: the segment's classes' B boxes (sg.map of them)
               const uint32_t tx =
                   grp ? (uint32_t)(DUAL >= 2 ? 2 : 1) * p.a_bytes + (uint32_t)sg.map * p.box_bytes
-                      : kRg ? p.a_bytes + (uint32_t)(sg.map == kRgWide ? 2 : 1) * (uint32_t)p.rg_n * 128u
+                      : kRg ? p.a_bytes + (uint32_t)(sg.map == kRgWide ? 2 : 1) * (uint32_t)p.rg_n * 128u *
+                                            (DUAL == 1 ? 2u : 1u)
                             : (PAIR ? 2u : 1u) * p.tx_bytes;
               mbar_expect_tx(&full_bar[st], tx);
             }
@@ -2134,10 +2135,11 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     ntiles = (long long)(q / 2) * q * p.n3;
     return launch<false, true, 0, false, 2>(p, ntiles, s);
   }
-  if (!swap && !dual && law == AAL_LAW_Q && q % 2 == 0 && 2 * bo <= 256 && rg_enabled()) {
+  if (!swap && law == AAL_LAW_Q && q % 2 == 0 && 2 * bo <= (dual ? 128 : 256) && rg_enabled()) {
     // Output-group pairs: the type's own segment x_t W(t, [k0, k0 + 2)) as
     // one MMA over both groups' columns, the two diagonal terms into their
-    // column ranges (half the tiles of one group each, and fewer MMAs)
+    // column ranges (half the tiles of one group each, and fewer MMAs); for
+    // the fused gate/up each of those is a gate MMA and an up MMA
     const int n = (int)(2 * bo);
     p.swap = 0;
     p.xr = 128;
@@ -2149,16 +2151,18 @@ static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long 
     p.rg_n = (int)bo;
     p.idesc = make_idesc(128, n, false, true);
     p.idesc_one = make_idesc(128, (int)bo, false, true);
-    if (!finish_plan(p, 0)) return AAL_ERR_UNSUPPORTED;
+    p.fuse_b = 0;
+    if (!finish_plan(p, dual ? 1 : 0)) return AAL_ERR_UNSUPPORTED;
     if (!map_kmajor(&p.mapA[0], X, q, 128)) return AAL_ERR_UNSUPPORTED;
     if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    if (dual && !map_mnmajor(&p.mapB[1], *Wu, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
     p.b_merged = 0;  // a diagonal segment loads only its group's atoms
     if (!out_map(p, Y, q)) return AAL_ERR_UNSUPPORTED;
     p.n1 = (int)((p.Mq + 127) / 128);
     p.n2 = q;
     p.n3 = 1;
     ntiles = (long long)q * p.n1 * (q / 2);
-    return launch<false, true, 0, false, 1>(p, ntiles, s);
+    return dual ? launch<false, true, 1, false, 1>(p, ntiles, s) : launch<false, true, 0, false, 1>(p, ntiles, s);
   }
   if (!swap) {
     const int n = pick_n(bo, dual ? 128 : 256);

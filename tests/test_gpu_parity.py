@@ -334,7 +334,7 @@ def test_square_medium(law, q, n):
                                   "fwd_offset", "fwd_ragged_tokens", "fwd_swap_groups_offset",
                                   "swiglu_swap_48_rows", "fwd_swap_q2xq2", "fwd_group_pairs_q2",
                                   "fwd_group_pairs_48", "fwd_class_pairs_48_rows",
-                                  "fwd_class_pairs_q4"])
+                                  "fwd_class_pairs_q4", "swiglu_group_pairs"])
 def test_tensor_path_small_cases(case):
     T = TENSOR
     if case == "fwd_swap":
@@ -366,6 +366,9 @@ def test_tensor_path_small_cases(case):
         r = run_project("Q", 16, 16 * 48, 512, 16 * 80, "bf16", seq_len=16 * 48, offset=3, policy=T)
     elif case == "fwd_class_pairs_q4":  # 64 rows a type, 96-column groups
         r = run_project("Q", 4, 256, 256, 384, "bf16", seq_len=256, policy=T)
+    elif case == "swiglu_group_pairs":  # gate/up in output-group pairs, 160 rows a type (a partial block)
+        eh, ey, p = run_swiglu("Q", 8, 8 * 160, 512, 8 * 48, "bf16", seq_len=8 * 160, policy=T)
+        r = (max(eh, ey), p)
     else:  # tokens per class not a multiple of the 128-row tile
         r = run_project("Q", 4, 4 * 200, 256, 512, "bf16", seq_len=800, policy=T)
     assert r[0] <= TOL["bf16"] and r[1] == T, r
@@ -388,7 +391,7 @@ print("ok")
 _ONE_GROUP_CHILD = r"""
 import sys
 sys.path.insert(0, sys.argv[1]); sys.path.insert(0, sys.argv[1] + '/tests')
-from gpu_cases import TOL, run_project, run_square
+from gpu_cases import TOL, run_project, run_square, run_swiglu
 import associative_algebra_block_b200 as aal
 T = aal.AAL_PATH_TENSOR
 for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512, 1024, 256, 5),
@@ -397,6 +400,8 @@ for q, M, din, dout, seq, off in ((16, 2048, 2048, 768, 2048, 0), (8, 1024, 512,
     assert err <= TOL["bf16"] and p == T, (q, err, p)
 err, p = run_square("Q", 4, 512, "bf16", policy=T)
 assert err <= TOL["bf16"] and p == T, (err, p)
+eh, ey, p = run_swiglu("Q", 16, 2048, 2048, 768, "bf16", seq_len=2048, policy=T)
+assert max(eh, ey) <= TOL["bf16"] and p == T, (eh, ey, p)
 print("ok")
 """
 
