@@ -60,12 +60,12 @@ ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c4-explicit", "c2-explicit", "qwe
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
     # c5: captured at n = 16384 (--config c5-n16384), x 4 for n = 32768 (4 x the tiles and bytes)
-    ("c5", "square product"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 4 * (1080665000 + 504161024), "aal_tc.cu"),
-    ("c5-n16384", "square product"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 1080665000 + 504161024, "aal_tc.cu"),
-    ("c2", "gate_up"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 23676928 + 1593856, "aal_tc.cu"),
-    ("c2", "down"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 40182784 + 983552, "aal_tc.cu"),
-    ("c3", "gate_up"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 218685184 + 34296064, "aal_tc.cu"),
-    ("c3", "down"): ("5dc9d47604e9ea9aff6292b24457e0ea998bf34a6d9c1aea4c4b599d546a9f64", 151098624 + 8467712, "aal_tc.cu"),
+    ("c5", "square product"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 4 * (1080481000 + 505112064), "aal_tc.cu"),
+    ("c5-n16384", "square product"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 1080481000 + 505112064, "aal_tc.cu"),
+    ("c2", "gate_up"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 23673600 + 1102336, "aal_tc.cu"),
+    ("c2", "down"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 40182784 + 1170176, "aal_tc.cu"),
+    ("c3", "gate_up"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 220092416 + 34213632, "aal_tc.cu"),
+    ("c3", "down"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 151098368 + 8200448, "aal_tc.cu"),
     ("c2", "decode gate_up B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 4746240, "aal_decode.cu"),
     ("c2", "decode down B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 2385152, "aal_decode.cu"),
 }
