@@ -5,7 +5,7 @@
 // 128 x N fp32 accumulator in tensor memory (TMEM) that sums, over the
 // members a of a table entry S(t, k), the block products X_a W_ak (agihunt.info
 // digest, multiplication-table paragraph).  The K range of a tile is a list of
-// up to four "segments" (one per table member, or a merged contiguous range),
+// up to six "segments" (one per table member, or a merged contiguous range),
 // walked in 64-element chunks; each chunk is one TMA load of an A tile and a B
 // tile into shared memory and up to four tcgen05.mma instructions (K = 16
 // each) accumulating into TMEM.  Because the |S| products of a tile land in
@@ -24,10 +24,22 @@
 // applying SiLU(g)*u or adding into the destination; two epilogue warps share
 // each 32-lane quarter of TMEM and split its columns), and warp 13 decodes
 // the tiles into a shared-memory ring the other roles read.
-// Tiles are visited longest first: a tile's cost is the number of block
-// products in its table entry (1, 2 or 4 for the laws here, up to q for the
-// backward's diagonal blocks), and the persistent CTAs stride through the
-// cost-sorted list so that every CTA ends with the short tiles.
+// Schedules: up to 1024 tiles of unequal cost are assigned on the host
+// longest first to the least loaded CTA; launches with many tiles a CTA hand
+// them out through a counter in device memory (CTAs that run faster take
+// more); the rest stride through the tile list.
+// Sharing the term common to several outputs (Q_q): on the swapped layout a
+// tile holds 2-4 row types and their diagonal term is one MMA (class groups);
+// on the unswapped projection, the fused gate/up and the square product a
+// tile holds two output groups and the type's (row block's) own term spans
+// both (output-group pairs); with at most 64 rows a type two types share an
+// unswapped tile (class pairs).  Each such mode is compiled only into the
+// instantiations that use it (the MODE template parameter, compile-time flags).
+// The backward's few very long tiles can run as split-K pieces added by a
+// reduction kernel (with a caller workspace).
+// Every launch is a programmatic dependent launch: a CTA sets up while the
+// previous grid finishes and waits (griddepcontrol.wait) before its first
+// global access; the tile decoder, which reads only parameters, starts early.
 // Shared-memory stages and the two TMEM accumulator buffers are handed over
 // with mbarriers; every wait is bounded (2 s of global time) and on expiry the
 // kernel records AAL_ERR_DEVICE_TIMEOUT in the status word, lets in-flight
