@@ -33,18 +33,30 @@ struct RowTypes {
 
 // Row type of row r; -1 (and the bounds flag) for an explicit type outside
 // [0, q) or a negative position.
-__device__ __forceinline__ int row_type(const RowTypes& rt, long long r) {
+// It is split into the load of the stored value (explicit type or position;
+// nothing for position types) and its decoding, so that a thread can issue
+// the loads of several rows before any check: a check may set the device
+// status, and a load after that store cannot be moved ahead of it.
+__device__ __forceinline__ long long row_type_raw(const RowTypes& rt, long long r) {
+  if (rt.kind == kTypesExplicit) return rt.types[r];
+  if (rt.kind == kTypesPositions64) return rt.positions[r];
+  return 0;
+}
+
+__device__ __forceinline__ int row_type_decode(const RowTypes& rt, long long r, long long raw) {
   if (rt.kind == kTypesPosition) {
     return (int)(((r % rt.seq_len) + rt.pos_offset) % rt.q);
   }
   if (rt.kind == kTypesExplicit) {
-    int t = rt.types[r];
-    if (t < 0 || t >= rt.q) { flag_device_error(kDevBounds); return -1; }
-    return t;
+    if (raw < 0 || raw >= rt.q) { flag_device_error(kDevBounds); return -1; }
+    return (int)raw;
   }
-  long long p = rt.positions[r];
-  if (p < 0) { flag_device_error(kDevBounds); return -1; }
-  return (int)(p % rt.q);
+  if (raw < 0) { flag_device_error(kDevBounds); return -1; }
+  return (int)(raw % rt.q);
+}
+
+__device__ __forceinline__ int row_type(const RowTypes& rt, long long r) {
+  return row_type_decode(rt, r, row_type_raw(rt, r));
 }
 
 // Membership a in S(t, k) of the multiplication table.

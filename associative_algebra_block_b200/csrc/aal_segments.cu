@@ -12,7 +12,12 @@
 // segment.  The tcgen05
 // kernel then runs in segment mode and its epilogue writes every output row
 // back to its original place.  No host synchronisation: the tile count stays
-// on the device and tiles past it are empty.
+// on the device and tiles past it are empty.  The launches form one chain of
+// programmatic dependent launches: each kernel lets the next one be launched
+// as soon as it starts, and waits for its predecessor's results before it
+// reads or writes anything, so the launch latencies overlap the work.
+#include <utility>
+
 #include "aal_internal.h"
 
 namespace aal {
@@ -21,6 +26,7 @@ namespace seg {
 constexpr int kThreads = 256;
 constexpr int kRowsPerBlock = 4096;
 constexpr int kMaxQ = 256;
+constexpr int kPerThread = kRowsPerBlock / kThreads;  // rows of a histogram / scatter thread
 
 struct Layout {
   size_t blk, counts, tiles, perm, xg, hg, total;
@@ -29,6 +35,28 @@ struct Layout {
 };
 
 static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Start of every kernel of the chain: release the next launch, then wait
+// until the previous grid has finished and its writes are visible.
+__device__ __forceinline__ void chain_enter() {
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... Exp, typename... Act>
+static cudaError_t launch_chained(void (*kernel)(Exp...), unsigned grid, unsigned block, cudaStream_t s,
+                                  Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
+}
 
 // Workspace of a call over ``rows`` rows gathering w1 columns (and w2 more
 // for a SwiGLU's hidden activation).
@@ -53,17 +81,85 @@ static Layout layout(int q, long long rows, long long w1, long long w2) {
   return L;
 }
 
+// Warp-aggregated claim on the per-type counters c (shared memory): the
+// lanes holding one type share a single atomic add.  Returns the lane's place
+// among the claims (its old counter value plus its rank among those lanes),
+// or -1 for t < 0.  All 32 lanes of the warp call it together.
+__device__ __forceinline__ int claim(int* c, int t) {
+  const unsigned peers = __match_any_sync(0xffffffffu, t);
+  const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
+  int base = 0;
+  if (t >= 0 && lane == leader) base = atomicAdd(&c[t], __popc(peers));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  return t >= 0 ? base + __popc(peers & ((1u << lane) - 1u)) : -1;
+}
+
+// Types of rows r0 + u * kStride + threadIdx.x (u < N; -1 at and past row
+// r0 + nr): every load is issued before any type is decoded and checked.
+template <int N, int kStride>
+__device__ __forceinline__ void load_types(const RowTypes& rt, long long r0, int nr, int (&ty)[N]) {
+  long long raw[N];
+#pragma unroll
+  for (int u = 0; u < N; ++u) {
+    const int i = u * kStride + (int)threadIdx.x;
+    raw[u] = i < nr ? row_type_raw(rt, r0 + i) : 0;
+  }
+#pragma unroll
+  for (int u = 0; u < N; ++u) {
+    const int i = u * kStride + (int)threadIdx.x;
+    ty[u] = i < nr ? row_type_decode(rt, r0 + i, raw[u]) : -1;
+  }
+}
+
+// Segment starts seg[t] and tile-table starts tst[t] (exclusive prefix sums
+// of the type counts cnt and of their 128-row tile counts), seg[q] and tst[q]
+// the totals; the tile total also goes to counts[q] and the row total to
+// counts[q + 1].  Run by warp 0: lane l
+// takes a run of ceil(q / 32) types, and a shuffle scan joins the runs.
+__device__ __forceinline__ void scan_starts(const int* cnt, int q, int* seg, int* tst, int* counts) {
+  const int lane = threadIdx.x & 31, per = (q + 31) / 32, a = lane * per, b = a + per < q ? a + per : q;
+  int sr = 0, nt = 0;
+  for (int t = a; t < b; ++t) {
+    sr += cnt[t];
+    nt += (cnt[t] + 127) / 128;
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int s2 = __shfl_up_sync(0xffffffffu, sr, o), n2 = __shfl_up_sync(0xffffffffu, nt, o);
+    if (lane >= o) {
+      sr += s2;
+      nt += n2;
+    }
+  }
+  int s0 = __shfl_up_sync(0xffffffffu, sr, 1), n0 = __shfl_up_sync(0xffffffffu, nt, 1);
+  if (lane == 0) s0 = n0 = 0;
+  for (int t = a; t < b; ++t) {
+    seg[t] = s0;
+    tst[t] = n0;
+    s0 += cnt[t];
+    n0 += (cnt[t] + 127) / 128;
+  }
+  if (lane == 31) {
+    seg[q] = sr;
+    tst[q] = nt;
+    counts[q] = nt;  // the tile count the tcgen05 kernel reads
+    counts[q + 1] = sr;
+  }
+}
+
 // 1. per-block histogram of the row types (rows with an invalid type are
 //    left out; row_type records the bounds error)
 __global__ void __launch_bounds__(kThreads) k_seg_hist(RowTypes rt, long long rows, int q, int* blk) {
+  chain_enter();
   __shared__ int c[kMaxQ];
   for (int i = threadIdx.x; i < q; i += kThreads) c[i] = 0;
   __syncthreads();
   const long long r0 = (long long)blockIdx.x * kRowsPerBlock;
-  for (int i = threadIdx.x; i < kRowsPerBlock && r0 + i < rows; i += kThreads) {
-    const int t = row_type(rt, r0 + i);
-    if (t >= 0) atomicAdd(&c[t], 1);
-  }
+  const int nr = (int)(rows - r0 < kRowsPerBlock ? rows - r0 : kRowsPerBlock);
+  int ty[kPerThread];
+  load_types<kPerThread, kThreads>(rt, r0, nr, ty);
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) claim(c, ty[u]);
   __syncthreads();
   for (int i = threadIdx.x; i < q; i += kThreads) blk[(long long)blockIdx.x * q + i] = c[i];
 }
@@ -72,6 +168,7 @@ __global__ void __launch_bounds__(kThreads) k_seg_hist(RowTypes rt, long long ro
 //    offsets (in place of the histogram), and the tile table
 __global__ void __launch_bounds__(kThreads) k_seg_scan(long long G, int q, int* blk, int* counts,
                                                        int4* tiles) {
+  chain_enter();
   __shared__ int tot[kMaxQ];
   __shared__ int seg[kMaxQ + 1];
   __shared__ int tst[kMaxQ + 1];
@@ -81,15 +178,7 @@ __global__ void __launch_bounds__(kThreads) k_seg_scan(long long G, int q, int* 
     tot[t] = s;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    seg[0] = 0;
-    tst[0] = 0;
-    for (int t = 0; t < q; ++t) {
-      seg[t + 1] = seg[t] + tot[t];
-      tst[t + 1] = tst[t] + (tot[t] + 127) / 128;
-    }
-    counts[q] = tst[q];  // the tile count the tcgen05 kernel reads
-  }
+  if (threadIdx.x < 32) scan_starts(tot, q, seg, tst, counts);
   __syncthreads();
   for (int t = threadIdx.x; t < q; t += kThreads) {
     int run = seg[t];
@@ -108,42 +197,41 @@ __global__ void __launch_bounds__(kThreads) k_seg_scan(long long G, int q, int* 
 //    records it
 __global__ void __launch_bounds__(kThreads) k_seg_scatter(RowTypes rt, long long rows, int q, const int* blk,
                                                           int* perm) {
+  chain_enter();
   __shared__ int cur[kMaxQ];
   for (int i = threadIdx.x; i < q; i += kThreads) cur[i] = blk[(long long)blockIdx.x * q + i];
   __syncthreads();
   const long long r0 = (long long)blockIdx.x * kRowsPerBlock;
   const int nr = (int)(rows - r0 < kRowsPerBlock ? rows - r0 : kRowsPerBlock);
-  for (int i = threadIdx.x; i < nr; i += kThreads) {
-    const int t = row_type(rt, r0 + i);
-    if (t >= 0) perm[atomicAdd(&cur[t], 1)] = (int)(r0 + i);
+  int ty[kPerThread];
+  load_types<kPerThread, kThreads>(rt, r0, nr, ty);
+#pragma unroll
+  for (int u = 0; u < kPerThread; ++u) {
+    const int d = claim(cur, ty[u]);
+    if (d >= 0) perm[d] = (int)(r0 + u * kThreads + threadIdx.x);
   }
 }
 
 // 1-3 in one block, for calls whose rows all fit one block of the histogram:
 // histogram, segment starts, tile table and permutation without leaving the
-// CTA (one launch instead of three).
+// CTA (one launch instead of three).  Each thread keeps its rows' types in
+// registers between the two passes.
 constexpr int kSmallThreads = 1024;
+constexpr int kSmallPer = kRowsPerBlock / kSmallThreads;
 __global__ void __launch_bounds__(kSmallThreads) k_seg_sort_small(RowTypes rt, long long rows, int q, int* counts,
                                                                   int4* tiles, int* perm) {
+  chain_enter();
   __shared__ int c[kMaxQ];
   __shared__ int seg[kMaxQ + 1];
   __shared__ int tst[kMaxQ + 1];
   for (int i = threadIdx.x; i < q; i += kSmallThreads) c[i] = 0;
   __syncthreads();
-  for (long long r = threadIdx.x; r < rows; r += kSmallThreads) {
-    const int t = row_type(rt, r);
-    if (t >= 0) atomicAdd(&c[t], 1);
-  }
+  int ty[kSmallPer];
+  load_types<kSmallPer, kSmallThreads>(rt, 0, (int)rows, ty);
+#pragma unroll
+  for (int u = 0; u < kSmallPer; ++u) claim(c, ty[u]);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    seg[0] = 0;
-    tst[0] = 0;
-    for (int t = 0; t < q; ++t) {
-      seg[t + 1] = seg[t] + c[t];
-      tst[t + 1] = tst[t] + (c[t] + 127) / 128;
-    }
-    counts[q] = tst[q];
-  }
+  if (threadIdx.x < 32) scan_starts(c, q, seg, tst, counts);
   __syncthreads();
   for (int t = threadIdx.x; t < q; t += kSmallThreads) {
     counts[t] = c[t];
@@ -152,30 +240,37 @@ __global__ void __launch_bounds__(kSmallThreads) k_seg_sort_small(RowTypes rt, l
     c[t] = seg[t];  // now the next free place of type t
   }
   __syncthreads();
-  for (long long r = threadIdx.x; r < rows; r += kSmallThreads) {
-    const int t = row_type(rt, r);
-    if (t >= 0) perm[atomicAdd(&c[t], 1)] = (int)r;
+#pragma unroll
+  for (int u = 0; u < kSmallPer; ++u) {
+    const int d = claim(c, ty[u]);
+    if (d >= 0) perm[d] = (int)(threadIdx.x + u * kSmallThreads);
   }
 }
 
 // 4. the gathered copy: row d of Xg is row perm[d] of X (one warp per row,
-//    16-byte vectors; rows past the sorted count are left alone)
-__global__ void __launch_bounds__(kThreads) k_seg_gather(const int* counts, int q, const int* perm,
-                                                         const __nv_bfloat16* X, long long ldx, int cols,
-                                                         __nv_bfloat16* Xg, long long ldg, long long rows) {
-  __shared__ int s_total;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int t = 0; t < q; ++t) n += counts[t];
-    s_total = n;
-  }
-  __syncthreads();
+//    16-byte vectors, kGatherBatch of them per lane loaded before any is
+//    stored; rows past the sorted count are left alone)
+constexpr int kGatherBatch = 8;
+__global__ void __launch_bounds__(kThreads) k_seg_gather(const int* __restrict__ counts, int q,
+                                                         const int* __restrict__ perm,
+                                                         const __nv_bfloat16* __restrict__ X, long long ldx, int cols,
+                                                         __nv_bfloat16* __restrict__ Xg, long long ldg, long long rows) {
+  chain_enter();
+  const int total = counts[q + 1];  // rows with a valid type
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nv = cols >> 3;
-  for (long long d = (long long)blockIdx.x * (kThreads / 32) + warp; d < rows && d < s_total;
+  for (long long d = (long long)blockIdx.x * (kThreads / 32) + warp; d < rows && d < total;
        d += (long long)gridDim.x * (kThreads / 32)) {
-    const uint4* src = reinterpret_cast<const uint4*>(X + (long long)perm[d] * ldx);
-    uint4* out = reinterpret_cast<uint4*>(Xg + d * ldg);
-    for (int v = lane; v < nv; v += 32) out[v] = src[v];
+    const uint4* __restrict__ src = reinterpret_cast<const uint4*>(X + (long long)perm[d] * ldx);
+    uint4* __restrict__ out = reinterpret_cast<uint4*>(Xg + d * ldg);
+    for (int v0 = lane; v0 < nv; v0 += 32 * kGatherBatch) {
+      uint4 r[kGatherBatch];
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u)
+        if (v0 + 32 * u < nv) r[u] = src[v0 + 32 * u];
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u)
+        if (v0 + 32 * u < nv) out[v0 + 32 * u] = r[u];
+    }
   }
 }
 
@@ -204,19 +299,22 @@ static aal_status seg_prepare(int q, const RowTypes& rt, long long rows, const a
   int4* tiles = (int4*)(ws + L.tiles);
   int* perm = (int*)(ws + L.perm);
   __nv_bfloat16* Xg = (__nv_bfloat16*)(ws + L.xg);
+  cudaError_t e;
   if (L.G == 1) {
-    k_seg_sort_small<<<1, kSmallThreads, 0, s>>>(rt, rows, q, counts, tiles, perm);
+    e = launch_chained(k_seg_sort_small, 1, kSmallThreads, s, rt, rows, q, counts, tiles, perm);
   } else {
-    k_seg_hist<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk);
-    k_seg_scan<<<1, seg::kThreads, 0, s>>>(L.G, q, blk, counts, tiles);
-    k_seg_scatter<<<(unsigned)L.G, seg::kThreads, 0, s>>>(rt, rows, q, blk, perm);
+    e = launch_chained(k_seg_hist, (unsigned)L.G, seg::kThreads, s, rt, rows, q, blk);
+    if (e == cudaSuccess) e = launch_chained(k_seg_scan, 1, seg::kThreads, s, L.G, q, blk, counts, tiles);
+    if (e == cudaSuccess) e = launch_chained(k_seg_scatter, (unsigned)L.G, seg::kThreads, s, rt, rows, q,
+                                             (const int*)blk, perm);
   }
   const long long gb = (rows + seg::kThreads / 32 - 1) / (seg::kThreads / 32);
-  k_seg_gather<<<(unsigned)(gb < 4096 ? gb : 4096), seg::kThreads, 0, s>>>(counts, q, perm,
-                                                                          (const __nv_bfloat16*)X.ptr, X.ld,
-                                                                          (int)X.cols, Xg, X.cols, rows);
+  if (e == cudaSuccess)
+    e = launch_chained(k_seg_gather, (unsigned)(gb < 4096 ? gb : 4096), seg::kThreads, s, (const int*)counts, q,
+                       (const int*)perm, (const __nv_bfloat16*)X.ptr, X.ld, (int)X.cols, Xg, (long long)X.cols,
+                       rows);
   note_launch(L.G == 1 ? 2 : 4);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(e);
 }
 
 // Common eligibility of the segment path (before anything is launched).

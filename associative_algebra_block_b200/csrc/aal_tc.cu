@@ -582,6 +582,34 @@ constexpr int kRgWide = 0x40, kRgNarrow = 0x20;
 // X_ig W_gg) and its rows are plain rows of X and Z.
 __device__ __forceinline__ void describe_rg(const Params& p, int tile, TileDesc& d) {
   const int npair = p.q >> 1;
+  if (p.seg_mode) {
+    // segment mode: entry j of the tile table (type t, gathered rows
+    // [e.y, e.z)) and output groups 2 kp, 2 kp + 1
+    const int j = tile / npair, k0 = 2 * (tile - j * npair);
+    d.nseg = 0;
+    d.a_c1 = 0;
+    d.b_f = k0 * p.bo;
+    d.b_c1 = 0;
+    d.rstride = 1;
+    d.roff = 0;
+    d.cbase = d.b_f;
+    d.vlo = 0;
+    d.vhi = INT_MAX;
+    if (j >= *(volatile const int*)p.seg_count) {  // past the table: an empty tile
+      d.a_f = 0;
+      d.rbase = 0;
+      d.rlimit = 0;
+      return;
+    }
+    const int4 e = p.seg_tiles[j];
+    add_seg(d, e.x * p.bi, p.bi, 0, kRgWide);
+    for (int g = 0; g < 2; ++g)
+      if (k0 + g != e.x) add_seg(d, (k0 + g) * p.bi, p.bi, 0, kRgNarrow | g);
+    d.a_f = e.y;
+    d.rbase = e.y;
+    d.rlimit = e.z;
+    return;
+  }
   const int kp = tile % npair, r = tile / npair, i1 = r % p.n1, c = r / p.n1;
   const bool sq = p.op == OP_SQUARE;
   const int k0 = 2 * kp, t = sq ? c : type_of_class(p, c);
@@ -2283,6 +2311,33 @@ aal_status tc_project_seg(int law, int q, long long rows, const aal_mat& Xg, con
   if (copy) {
     p.seg_copy = (__nv_bfloat16*)copy->ptr;
     p.ld_copy = copy->ld;
+  }
+  if (law == AAL_LAW_Q && q % 2 == 0 && 2 * bo <= (dual ? 128 : 256) && rg_enabled()) {
+    // output-group pairs, as on the strided path: tile (j, kp) is table
+    // entry j against output groups 2 kp and 2 kp + 1
+    const int n = (int)(2 * bo);
+    p.swap = 0;
+    p.xr = 128;
+    p.wn = n;
+    p.n_mma = n;
+    p.a_rows = 128;
+    p.b_rows = n;
+    p.b_aw = bo % 64 == 0 ? 64 : 16;
+    p.rg_n = (int)bo;
+    p.idesc = make_idesc(128, n, false, true);
+    p.idesc_one = make_idesc(128, (int)bo, false, true);
+    p.fuse_b = 0;
+    if (!finish_plan(p, dual ? 1 : 0)) return AAL_ERR_UNSUPPORTED;
+    if (!map_kmajor(&p.mapA[0], Xg, 1, 128)) return AAL_ERR_UNSUPPORTED;
+    if (!map_mnmajor(&p.mapB[0], Wg, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    if (dual && !map_mnmajor(&p.mapB[1], *Wu, 1, p.b_aw)) return AAL_ERR_UNSUPPORTED;
+    p.b_merged = 0;  // a diagonal segment loads only its group's atoms
+    if (!out_map(p, Y, 1)) return AAL_ERR_UNSUPPORTED;
+    p.n1 = 1;
+    p.n2 = q;
+    p.n3 = 1;
+    const long long ntiles = (long long)tmax * (q / 2);
+    return dual ? launch<false, true, 1, false, 1>(p, ntiles, s) : launch<false, true, 0, false, 1>(p, ntiles, s);
   }
   const int n = pick_n(bo, dual ? 128 : 256);
   if (!n) return AAL_ERR_UNSUPPORTED;

@@ -402,6 +402,11 @@ err, p = run_square("Q", 4, 512, "bf16", policy=T)
 assert err <= TOL["bf16"] and p == T, (err, p)
 eh, ey, p = run_swiglu("Q", 16, 2048, 2048, 768, "bf16", seq_len=2048, policy=T)
 assert max(eh, ey) <= TOL["bf16"] and p == T, (eh, ey, p)
+# segment mode (explicit types through the workspace)
+err, p = run_project("Q", 16, 2048, 2048, 768, "bf16", explicit=True, seed=5, ws=True, policy=T)
+assert err <= TOL["bf16"] and p == T, (err, p)
+eh, ey, p = run_swiglu("Q", 16, 2048, 2048, 768, "bf16", seq_len=2047, seed=6, ws=True, policy=T)
+assert max(eh, ey) <= TOL["bf16"] and p == T, (eh, ey, p)
 print("ok")
 """
 
@@ -592,6 +597,8 @@ def test_tcgen05_wait_that_runs_out_reports_timeout_and_returns():
     ("Q", 8, 1003, 256, 512, 37, False),           # ragged rows and sequences
     ("Q", 32, 333, 4096, 2048, None, True),        # few rows per type (partial tiles)
     ("Q", 4, 7, 128, 256, None, True),             # fewer rows than types
+    ("Q", 5, 1500, 320, 640, None, True),          # odd q: one output group a tile
+    ("Q", 4, 1000, 256, 1024, None, True),         # groups too wide to pair
 ])
 def test_explicit_and_ragged_types_tensor_path(law, q, M, din, dout, seq_len, explicit):
     err, path = run_project(law, q, M, din, dout, "bf16", seq_len=seq_len, explicit=explicit,
