@@ -93,6 +93,56 @@ void* current_workspace(uint64_t* bytes) {
   return t_ws;
 }
 
+// A second stream of this host thread on each device it uses, with the events
+// that fork it from the caller's stream and join it back.  The fork and join
+// are an event record and a stream wait, so they work the same way while the
+// caller's stream is being captured into a CUDA graph (the second stream then
+// joins the capture).
+struct SideStream {
+  int dev = -1;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static thread_local SideStream t_side[8];
+
+// The side stream, ordered after everything queued on ``s`` so far; null if
+// it cannot be had (the caller then stays on ``s``).
+static cudaStream_t fork_side(cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  SideStream* ss = nullptr;
+  for (SideStream& e : t_side)
+    if (e.dev == dev) { ss = &e; break; }
+  if (!ss) {
+    for (SideStream& e : t_side)
+      if (e.dev < 0) { ss = &e; break; }
+    if (!ss) return nullptr;
+    if (cudaStreamCreateWithFlags(&ss->s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&ss->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss->join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(ss->s);
+      if (ss->fork) cudaEventDestroy(ss->fork);
+      *ss = SideStream();
+      return nullptr;
+    }
+    ss->dev = dev;
+  }
+  if (cudaEventRecord(ss->fork, s) != cudaSuccess) return nullptr;
+  if (cudaStreamWaitEvent(ss->s, ss->fork, 0) != cudaSuccess) return nullptr;
+  return ss->s;
+}
+
+// Orders ``s`` after everything queued on the side stream ``side`` so far.
+static aal_status join_side(cudaStream_t s, cudaStream_t side) {
+  for (SideStream& e : t_side)
+    if (e.s == side) {
+      if (cudaEventRecord(e.join, side) != cudaSuccess || cudaStreamWaitEvent(s, e.join, 0) != cudaSuccess)
+        return AAL_ERR_CUDA;
+      return AAL_OK;
+    }
+  return AAL_ERR_CUDA;
+}
+
 }  // namespace aal
 
 using namespace aal;
@@ -181,19 +231,48 @@ aal_status aal_project_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_m
   cudaStream_t s = (cudaStream_t)stream;
   RowTypes rt = make_types(rule, q);
   int paths = 0;
+  // Small problems run dX (on s) and dW (on a side stream) side by side, each
+  // on half of the SMs, with the split-K partials of dW placed after dX's in
+  // the workspace.
+  cudaStream_t sw = s;
+  void* const ws0 = t_ws;
+  const uint64_t ws0_bytes = t_ws_bytes;
+  int64_t dw_off = 0;
+  if (want_dx && want_dw && M > 0 && t_policy != AAL_PATH_GENERAL && X.dtype == AAL_BF16 &&
+      tc_bwd_side_by_side(M, din, dout)) {
+    cudaStream_t side = fork_side(s);
+    if (side) {
+      sw = side;
+      set_sm_share(device_sms() / 2);
+      int64_t a = 0, b = 0;
+      tc_bwd_split_parts(law, q, M, din, dout, &a, &b);
+      dw_off = (a + 255) & ~(int64_t)255;
+    }
+  }
+  aal_status st = AAL_OK;
   if (want_dx && M > 0 && din > 0) {
-    aal_status st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dY, W, dX, 0, s); },
-                             [&] { return simt_project_bwd_dx(law, q, rt, dY, W, dX, s); });
-    if (st != AAL_OK) return st;
-    paths |= 1 << t_last_path;
+    st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_project_bwd_dx(law, q, rt, M, dY, W, dX, 0, s); },
+                  [&] { return simt_project_bwd_dx(law, q, rt, dY, W, dX, s); });
+    if (st == AAL_OK) paths |= 1 << t_last_path;
   }
-  if (want_dw && din > 0 && dout > 0) {
-    aal_status st =
-        dispatch(AAL_KERNEL_BWD_DW, s, [&] { return tc_project_bwd_dw(law, q, rt, M, X, dY, dW, accumulate_dW, s); },
-                 [&] { return simt_project_bwd_dw(law, q, rt, X, dY, dW, accumulate_dW, s); });
-    if (st != AAL_OK) return st;
-    paths |= 1 << t_last_path;
+  if (st == AAL_OK && want_dw && din > 0 && dout > 0) {
+    if (sw != s) {
+      const bool fits = ws0 && (uint64_t)dw_off < ws0_bytes;
+      t_ws = fits ? (char*)ws0 + dw_off : nullptr;
+      t_ws_bytes = fits ? ws0_bytes - (uint64_t)dw_off : 0;
+    }
+    st = dispatch(AAL_KERNEL_BWD_DW, sw, [&] { return tc_project_bwd_dw(law, q, rt, M, X, dY, dW, accumulate_dW, sw); },
+                  [&] { return simt_project_bwd_dw(law, q, rt, X, dY, dW, accumulate_dW, sw); });
+    t_ws = ws0;
+    t_ws_bytes = ws0_bytes;
+    if (st == AAL_OK) paths |= 1 << t_last_path;
   }
+  if (sw != s) {
+    set_sm_share(0);
+    const aal_status sj = join_side(s, sw);  // always: a capture must end joined
+    if (st == AAL_OK) st = sj;
+  }
+  if (st != AAL_OK) return st;
   if (paths) note_path((paths & (1 << AAL_PATH_GENERAL)) ? AAL_PATH_GENERAL : AAL_PATH_TENSOR);
   return AAL_OK;
 }
@@ -221,28 +300,64 @@ aal_status aal_swiglu_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_ma
   cudaStream_t s = (cudaStream_t)stream;
   RowTypes rt = make_types(rule, q);
   int paths = 0;
-  aal_status st;
+  aal_status st = AAL_OK;
   auto note = [&] { paths |= 1 << t_last_path; };
+  // weight gradient i: dWd (needs only H and dY), dWg, dWu
+  const aal_mat* dw_in[3][3] = {{&H, &dY, &dWd}, {&X, &dG, &dWg}, {&X, &dU, &dWu}};
+  auto weight_grad = [&](int i, cudaStream_t on) {
+    const aal_mat &A = *dw_in[i][0], &B = *dw_in[i][1], &O = *dw_in[i][2];
+    aal_status e = dispatch(AAL_KERNEL_BWD_DW, on, [&] { return tc_project_bwd_dw(law, q, rt, M, A, B, O, 0, on); },
+                            [&] { return simt_project_bwd_dw(law, q, rt, A, B, O, 0, on); });
+    if (e == AAL_OK) note();
+    return e;
+  };
   if (M > 0) {
     // 1. the gate and up pre-activations, recomputed
     st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, X, Wg, G, s); },
                   [&] { return simt_project(law, q, rt, X, Wg, G, s); });
-    if (st != AAL_OK) return st;
-    note();
-    st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, X, Wu, U, s); },
-                  [&] { return simt_project(law, q, rt, X, Wu, U, s); });
-    if (st != AAL_OK) return st;
-    note();
+    if (st == AAL_OK) {
+      note();
+      st = dispatch(AAL_KERNEL_PROJECT, s, [&] { return tc_project(law, q, rt, M, X, Wu, U, s); },
+                    [&] { return simt_project(law, q, rt, X, Wu, U, s); });
+    }
+    if (st == AAL_OK) note();
     // 2. dH = dY through the down projection's transposed table, and the
     //    SiLU' chain: dG = dH u silu'(g), dU = dH silu(g)
-    st = dispatch(AAL_KERNEL_SWIGLU_BWD, s,
-                  [&] { return tc_swiglu_bwd_dh(law, q, rt, M, dY, Wd, G, U, dG, dU, s); },
-                  [&] {
-                    aal_status e = simt_project_bwd_dx(law, q, rt, dY, Wd, dG, s);
-                    return e != AAL_OK ? e : simt_swiglu_bwd_act(q, rt, G, U, dG, dU, s);
-                  });
-    if (st != AAL_OK) return st;
-    note();
+    if (st == AAL_OK)
+      st = dispatch(AAL_KERNEL_SWIGLU_BWD, s,
+                    [&] { return tc_swiglu_bwd_dh(law, q, rt, M, dY, Wd, G, U, dG, dU, s); },
+                    [&] {
+                      aal_status e = simt_project_bwd_dx(law, q, rt, dY, Wd, dG, s);
+                      return e != AAL_OK ? e : simt_swiglu_bwd_act(q, rt, G, U, dG, dU, s);
+                    });
+    if (st == AAL_OK) note();
+  }
+  if (st != AAL_OK) return st;
+  // Small problems run the four launches after dH side by side, every launch
+  // on half of the SMs: dX then dWu on the caller's stream, dWd then dWg on a
+  // side stream, whose split-K partials follow the caller stream's in the
+  // workspace.
+  cudaStream_t sw = s;
+  if (M > 0 && t_policy != AAL_PATH_GENERAL && X.dtype == AAL_BF16 && tc_bwd_side_by_side(M, D, F)) {
+    cudaStream_t side = fork_side(s);
+    if (side) {
+      sw = side;
+      set_sm_share(device_sms() / 2);
+      int64_t dx = 0, dw = 0;
+      tc_bwd_split_parts(law, q, M, D, F, &dx, &dw);
+      const int64_t off = ((dx > dw ? dx : dw) + 255) & ~(int64_t)255;
+      void* const ws0 = t_ws;
+      const uint64_t ws0_bytes = t_ws_bytes;
+      const bool fits = ws0 && (uint64_t)off < ws0_bytes;
+      t_ws = fits ? (char*)ws0 + off : nullptr;
+      t_ws_bytes = fits ? ws0_bytes - (uint64_t)off : 0;
+      st = weight_grad(0, sw);
+      if (st == AAL_OK) st = weight_grad(1, sw);
+      t_ws = ws0;
+      t_ws_bytes = ws0_bytes;
+    }
+  }
+  if (st == AAL_OK && M > 0) {
     // 3. dX = dG Wg^T + dU Wu^T over the table: one tensor-core launch with
     //    both products in the same accumulator, else two general passes
     st = dispatch(AAL_KERNEL_BWD_DX, s, [&] { return tc_swiglu_bwd_dx(law, q, rt, M, dG, Wg, dU, Wu, dX, s); },
@@ -250,18 +365,18 @@ aal_status aal_swiglu_bwd(int32_t law, int32_t q, aal_row_type_rule rule, aal_ma
                     aal_status e = simt_project_bwd_dx(law, q, rt, dG, Wg, dX, s);
                     return e != AAL_OK ? e : simt_project_bwd_dx(law, q, rt, dU, Wu, dX, s, 1);
                   });
-    if (st != AAL_OK) return st;
-    note();
+    if (st == AAL_OK) note();
   }
   // 4. weight gradients (zero when there are no rows)
-  const aal_mat* dw_in[3][3] = {{&X, &dG, &dWg}, {&X, &dU, &dWu}, {&H, &dY, &dWd}};
-  for (auto& t : dw_in) {
-    const aal_mat &A = *t[0], &B = *t[1], &O = *t[2];
-    st = dispatch(AAL_KERNEL_BWD_DW, s, [&] { return tc_project_bwd_dw(law, q, rt, M, A, B, O, 0, s); },
-                  [&] { return simt_project_bwd_dw(law, q, rt, A, B, O, 0, s); });
-    if (st != AAL_OK) return st;
-    note();
+  if (sw != s) {
+    if (st == AAL_OK) st = weight_grad(2, s);
+    set_sm_share(0);
+    const aal_status sj = join_side(s, sw);  // always: a capture must end joined
+    if (st == AAL_OK) st = sj;
+  } else {
+    for (int i = 0; i < 3 && st == AAL_OK; ++i) st = weight_grad(i, s);
   }
+  if (st != AAL_OK) return st;
   note_path((paths & (1 << AAL_PATH_GENERAL)) ? AAL_PATH_GENERAL : AAL_PATH_TENSOR);
   return AAL_OK;
 }
@@ -449,9 +564,8 @@ int64_t aal_workspace_size(int32_t call, int32_t law, int32_t q, aal_row_type_ru
   if (call == AAL_CALL_PROJECT_BWD || call == AAL_CALL_SWIGLU_BWD) {
     // split K of the heavy tiles (position rules on the tensor-core path only)
     if (seg_needed(rt, q, rows)) return 0;
-    const int64_t a = tc_bwd_split_bytes(law, q, rows, d_in, d_hidden);
-    const int64_t b = call == AAL_CALL_SWIGLU_BWD ? tc_bwd_split_bytes(law, q, rows, d_hidden, d_in) : 0;
-    return a > b ? a : b;
+    return call == AAL_CALL_SWIGLU_BWD ? tc_swiglu_bwd_split_bytes(law, q, rows, d_in, d_hidden)
+                                       : tc_bwd_split_bytes(law, q, rows, d_in, d_hidden);
   }
   if (!seg_needed(rt, q, rows)) return 0;
   return seg_workspace_bytes(q, rows, d_in, call == AAL_CALL_SWIGLU_FWD ? d_hidden : 0);

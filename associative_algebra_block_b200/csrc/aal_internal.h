@@ -146,6 +146,18 @@ void* current_workspace(uint64_t* bytes);
 // Workspace bytes the tensor-core backward of a projection W [din, dout]
 // uses to split its heavy Q_q tiles (0: no split for these sizes).
 int64_t tc_bwd_split_bytes(int law, int q, long long rows, long long din, long long dout);
+// Split-K workspace bytes of a projection backward's dX and dW launches at the
+// SM share in force.
+void tc_bwd_split_parts(int law, int q, long long rows, long long din, long long dout, int64_t* dx,
+                        int64_t* dw);
+// The same for a SwiGLU backward of X [rows, D] through a hidden width F.
+int64_t tc_swiglu_bwd_split_bytes(int law, int q, long long rows, long long D, long long F);
+// Whether a projection backward runs dX and dW side by side on two streams.
+bool tc_bwd_side_by_side(long long rows, long long din, long long dout);
+// SMs of the current device, and the share of them that the tensor-core
+// launches of this thread may use (0: all).
+int device_sms();
+void set_sm_share(int n);
 int64_t seg_workspace_bytes(int q, long long rows, long long w1, long long w2);
 aal_status seg_project_fwd(int law, int q, const RowTypes& rt, const aal_mat& X, const aal_mat& W,
                            const aal_mat& Y, void* ws, uint64_t ws_bytes, cudaStream_t s);

@@ -1584,11 +1584,20 @@ static uint32_t make_idesc(int m, int n, bool a_mn, bool b_mn) {
   return d;
 }
 
-static int num_sms() {
+// SM share of the launches this thread makes while it is set (0: all SMs):
+// two launches that run side by side on two streams take half of the GPU each.
+static thread_local int t_sm_share = 0;
+
+static int all_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n > 0 ? n : 148;
+}
+
+static int num_sms() {
+  const int n = all_sms();
+  return (t_sm_share > 0 && t_sm_share < n) ? t_sm_share : n;
 }
 
 static bool is_sm100() {
@@ -2059,6 +2068,9 @@ static void base_params(Params& p, int law, int q, const RowTypes& rt, long long
 
 using namespace tc;
 
+void set_sm_share(int n) { t_sm_share = n; }
+int device_sms() { return all_sms(); }
+
 // Projection and fused gate/up share the planning; ``Wu`` null -> projection.
 static aal_status tc_project_impl(int law, int q, const RowTypes& rt, long long rows,
                                   const aal_mat& X, const aal_mat& Wg, const aal_mat* Wu,
@@ -2477,12 +2489,65 @@ aal_status tc_swiglu_bwd_dh(int law, int q, const RowTypes& rt, long long rows, 
   return bwd_dx_impl(law, q, rt, rows, dY, Wd, dG, 0, &G, &U, &dU, s);
 }
 
-int64_t tc_bwd_split_bytes(int law, int q, long long rows, long long din, long long dout) {
-  if (law != AAL_LAW_Q || q < 2 || rows % q || din % q || dout % q) return 0;
+void tc_bwd_split_parts(int law, int q, long long rows, long long din, long long dout, int64_t* dx,
+                        int64_t* dw) {
+  *dx = *dw = 0;
+  if (law != AAL_LAW_Q || q < 2 || rows % q || din % q || dout % q) return;
   const long long bi = din / q, bo = dout / q;
-  if (bi % 16 || bo % 16) return 0;
-  const int64_t a = split_bytes(geom_dx(q, rows, bi, bo)), b = split_bytes(geom_dw(q, rows, bi, bo));
-  return a > b ? a : b;
+  if (bi % 16 || bo % 16) return;
+  *dx = split_bytes(geom_dx(q, rows, bi, bo));
+  *dw = split_bytes(geom_dw(q, rows, bi, bo));
+}
+
+// AAL_TC_SIDE_BY_SIDE=0 in the environment keeps a projection backward's dX
+// and dW launches one after the other on the caller's stream (read once).
+static bool side_by_side_enabled() {
+  static const int v = [] {
+    const char* e = getenv("AAL_TC_SIDE_BY_SIDE");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return v != 0;
+}
+
+bool tc_bwd_side_by_side(long long rows, long long din, long long dout) {
+  // small problems only: a few tiles a CTA, so that the launches' fixed
+  // start-up and drain overlap; larger ones fill the GPU one at a time
+  return side_by_side_enabled() && rows > 0 && din > 0 && dout > 0 &&
+         (double)rows * (double)din * (double)dout <= 8.6e9;
+}
+
+int64_t tc_bwd_split_bytes(int law, int q, long long rows, long long din, long long dout) {
+  int64_t a = 0, b = 0;
+  tc_bwd_split_parts(law, q, rows, din, dout, &a, &b);
+  int64_t need = a > b ? a : b;
+  if (tc_bwd_side_by_side(rows, din, dout)) {
+    // side by side: dX's partials first, dW's after them, each planned on half the SMs
+    const int keep = t_sm_share;
+    t_sm_share = all_sms() / 2;
+    tc_bwd_split_parts(law, q, rows, din, dout, &a, &b);
+    t_sm_share = keep;
+    const int64_t both = ((a + 255) & ~(int64_t)255) + b;
+    if (both > need) need = both;
+  }
+  return need;
+}
+
+int64_t tc_swiglu_bwd_split_bytes(int law, int q, long long rows, long long D, long long F) {
+  const int64_t a = tc_bwd_split_bytes(law, q, rows, D, F), b = tc_bwd_split_bytes(law, q, rows, F, D);
+  int64_t need = a > b ? a : b;
+  if (tc_bwd_side_by_side(rows, D, F)) {
+    // dX (gate + up) then dWu on the caller's stream, dWd then dWg on the
+    // side stream after them in the workspace, all planned on half the SMs
+    const int keep = t_sm_share;
+    t_sm_share = all_sms() / 2;
+    int64_t dx = 0, dw = 0, dx2 = 0, dwd = 0;
+    tc_bwd_split_parts(law, q, rows, D, F, &dx, &dw);
+    tc_bwd_split_parts(law, q, rows, F, D, &dx2, &dwd);
+    t_sm_share = keep;
+    const int64_t both = (((dx > dw ? dx : dw) + 255) & ~(int64_t)255) + (dw > dwd ? dw : dwd);
+    if (both > need) need = both;
+  }
+  return need;
 }
 
 aal_status tc_project_bwd_dw(int law, int q, const RowTypes& rt, long long rows, const aal_mat& X,

@@ -535,13 +535,13 @@ class SwigluFwdBwd:
             "bwd G recompute": (self.f_df, e * (M * D + D * F + M * F)),
             "bwd dH + SiLU'": (self.f_fd, e * (M * D + F * D + 4 * M * F)),
             "bwd dX (gate + up)": (2 * self.f_df, e * (2 * M * F + 2 * D * F + M * D)),
-            "bwd dWg": (self.f_df, e * (M * D + M * F + D * F)),
+            "bwd dWd": (self.f_fd, e * (M * F + M * D + F * D)),
         }[name]
 
     def timing_slots(self):
         return [("fwd gate_up", aal.AAL_KERNEL_GATE_UP), ("fwd down", aal.AAL_KERNEL_PROJECT),
                 ("bwd G recompute", aal.AAL_KERNEL_PROJECT), ("bwd dH + SiLU'", aal.AAL_KERNEL_SWIGLU_BWD),
-                ("bwd dX (gate + up)", aal.AAL_KERNEL_BWD_DX), ("bwd dWg", aal.AAL_KERNEL_BWD_DW)]
+                ("bwd dX (gate + up)", aal.AAL_KERNEL_BWD_DX), ("bwd dWd", aal.AAL_KERNEL_BWD_DW)]
 
     def group_names(self):
         return []
