@@ -279,6 +279,16 @@ AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat
  * same sum in another association order.  The dH step of aal_swiglu_bwd
  * (its SiLU' chain needs the whole sum) is never split.
  *
+ * Small backward problems (rows * d_in * d_hidden up to about 8.6e9) also
+ * run launches side by side: aal_project_bwd puts dW on a second stream of
+ * the calling host thread beside dX, and aal_swiglu_bwd puts dWd and dWg
+ * there beside dX and dWu, each launch on half of the SMs.  The second stream
+ * is forked from and joined back to the call's stream by event records and
+ * stream waits (so the call also captures into a CUDA graph), and the call's
+ * stream orders everything as before.  The second stream's partial sums sit
+ * after the first stream's in the workspace, and aal_workspace_size covers
+ * that layout.
+ *
  * aal_workspace_size: bytes the call needs for ``rows`` rows; call is
  * AAL_CALL_PROJECT_FWD (d_in = din, d_hidden unused), AAL_CALL_SWIGLU_FWD
  * (d_in = D, d_hidden = F), AAL_CALL_PROJECT_BWD (d_in = din, d_hidden =
@@ -399,6 +409,9 @@ AAL_API int32_t aal_version(void);
  *   AAL_DECODE_MMA=0         SIMT decode kernels instead of the tensor-core one.
  *   AAL_DECODE_TYPED=0       the cluster decode kernel for single-type batches.
  *   AAL_FFN_DECODE_FUSED=1   the one-launch FFN decode (default off: slower).
+ *   AAL_TC_SIDE_BY_SIDE=0    the backward calls keep every launch on the call's
+ *                            stream (default: small problems run their weight
+ *                            gradients on a second stream, see above).
  *   AAL_TEST_STALL=1         test hook: the tcgen05 kernel's MMA thread waits on
  *                            a barrier nothing arrives on until the bounded
  *                            wait runs out (AAL_ERR_DEVICE_TIMEOUT); read at
