@@ -60,12 +60,12 @@ ALL_CONFIGS = ("c2", "c3", "c4", "c4-swiglu", "c4-explicit", "c2-explicit", "qwe
 NCU_TRAFFIC = {
     # (workload, kernel): (sha256 of its source file, dram bytes per launch, source file)
     # c5: captured at n = 16384 (--config c5-n16384), x 4 for n = 32768 (4 x the tiles and bytes)
-    ("c5", "square product"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 4 * (1080481000 + 505112064), "aal_tc.cu"),
-    ("c5-n16384", "square product"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 1080481000 + 505112064, "aal_tc.cu"),
-    ("c2", "gate_up"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 23673600 + 1102336, "aal_tc.cu"),
-    ("c2", "down"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 40182784 + 1170176, "aal_tc.cu"),
-    ("c3", "gate_up"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 220092416 + 34213632, "aal_tc.cu"),
-    ("c3", "down"): ("31a57c235965c90dd093ebd631ef21156055b6c16ebf51e9bd231142c5cfb1e7", 151098368 + 8200448, "aal_tc.cu"),
+    ("c5", "square product"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 4 * (1080002560 + 505648896), "aal_tc.cu"),
+    ("c5-n16384", "square product"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 1080002560 + 505648896, "aal_tc.cu"),
+    ("c2", "gate_up"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 23672832 + 1167872, "aal_tc.cu"),
+    ("c2", "down"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 40182528 + 957696, "aal_tc.cu"),
+    ("c3", "gate_up"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 220005632 + 33688320, "aal_tc.cu"),
+    ("c3", "down"): ("4940aa66ebd5351af057bc357ab225b16a95a390d0adb3debcbe8e6d112cb530", 151123968 + 9446144, "aal_tc.cu"),
     ("c2", "decode gate_up B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 4746240, "aal_decode.cu"),
     ("c2", "decode down B=1"): ("9fa8764bed43c9a4cf4e245e9cc4941d4fa162ccbc70ebeb1c0c118a8dc7c3ea", 2385152, "aal_decode.cu"),
 }
