@@ -1,10 +1,14 @@
-// General CUDA path: one thread per output element, fp32 accumulation.
+// General CUDA path, fp32 accumulation.
 //
 // Serves every call for any shape the header allows: fp32 (the Q_2 fp32
-// workload), explicit row types, sequence lengths that are not a multiple of
-// q, and the ragged tail rows the tensor-core path leaves.  The loops follow
-// the table directly: output block (t, k) of a row of type t sums x_a W_ak
-// over a in S(t, k) (agihunt.info digest, multiplication-table paragraph).
+// workload), explicit row types without a workspace, sequence lengths that
+// are not a multiple of q, the backward with such rules, and shapes the
+// tensor-core path does not take.  The sums follow the table directly: output
+// block (t, k) of a row of type t sums x_a W_ak over a in S(t, k) (agihunt.info
+// digest, multiplication-table paragraph).  Projections and dX with at least
+// half a tile of rows, and every dW, run on shared-memory tiles that keep only
+// the rows each table entry applies to; small calls (decode rows) and the
+// SwiGLU and square-product kernels compute one output per thread.
 #include "aal_internal.h"
 
 namespace aal {
@@ -135,6 +139,213 @@ __global__ void k_bwd_dw(int law, int q, RowTypes rt, long long rows, const T* _
   st_elem(out, acc);
 }
 
+// Y (kDx false) or dX (kDx true) on tiles of 64 rows by up to 64 outputs of
+// one group g, 256 threads of 4 x 4 products.  For each group m of the
+// contraction the tile keeps the rows whose type t has the table entry (Y:
+// m in S(t, g); dX: g in S(t, m)), stages their operand slices 32 contraction
+// steps at a time beside the matching weight slice, and adds the products to
+// an accumulator in shared memory; the work follows the table row by row and
+// every weight element is read once per tile.
+//   Y:  A = X,  contraction group width L = bi, output group width G = bo,
+//       weight W[m*bi + c, g*bo + f]
+//   dX: A = dY, L = bo, G = bi, weight W[g*bi + f, m*bo + c]
+constexpr int kRtRows = 64, kRtOut = 64, kRtK = 32;
+template <typename T, bool kDx>
+__global__ void __launch_bounds__(256) k_rows_tiled(int law, int q, RowTypes rt, long long row_begin,
+                                                    long long rows, const T* __restrict__ A, long long lda,
+                                                    const T* __restrict__ W, long long ldw, T* __restrict__ O,
+                                                    long long ldo, int L, int G, int accumulate) {
+  __shared__ float acc_s[kRtRows][kRtOut + 1];
+  __shared__ float as[kRtRows][kRtK + 1];
+  __shared__ float bs[kRtOut][kRtK + 1];
+  __shared__ int s_t[kRtRows];
+  __shared__ int s_idx[kRtRows];
+  __shared__ unsigned s_mask[kRtRows / 32];
+  const int ot_per = (G + kRtOut - 1) / kRtOut;
+  const int g = (int)(blockIdx.x / (unsigned)ot_per);
+  const int o_lo = (int)(blockIdx.x - (unsigned)g * ot_per) * kRtOut;
+  const int no = G - o_lo < kRtOut ? G - o_lo : kRtOut;
+  const long long r0 = row_begin + (long long)blockIdx.y * kRtRows;
+  const int nr = (int)(rows - r0 < kRtRows ? rows - r0 : kRtRows);
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  for (int e = tid; e < kRtRows * (kRtOut + 1); e += 256) (&acc_s[0][0])[e] = 0.f;
+  if (tid < kRtRows) s_t[tid] = tid < nr ? row_type(rt, r0 + tid) : -1;
+  __syncthreads();
+  for (int m = 0; m < q; ++m) {
+    // the rows of the tile that take part in group m, packed in row order
+    if (tid < kRtRows) {
+      const int t = s_t[tid];
+      const bool keep = t >= 0 && (kDx ? in_table(law, t, m, g) : in_table(law, t, g, m));
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if ((tid & 31) == 0) s_mask[tid >> 5] = bal;
+    }
+    __syncthreads();
+    const unsigned m0 = s_mask[0], m1 = s_mask[1];
+    const int n = __popc(m0) + __popc(m1);
+    if (n > 0) {
+      if (tid < kRtRows) {
+        const unsigned mine = tid < 32 ? m0 : m1;
+        const int bit = tid & 31;
+        if ((mine >> bit) & 1u)
+          s_idx[(tid < 32 ? 0 : __popc(m0)) + __popc(mine & ((1u << bit) - 1u))] = tid;
+      }
+      __syncthreads();
+      float part[4][4] = {};
+      for (int c0 = 0; c0 < L; c0 += kRtK) {
+        const int nc = L - c0 < kRtK ? L - c0 : kRtK;
+        for (int e = tid; e < n * kRtK; e += 256) {
+          const int sl = e / kRtK, cc = e - sl * kRtK;
+          as[sl][cc] = cc < nc ? ld_elem(A + (r0 + s_idx[sl]) * lda + (long long)m * L + c0 + cc) : 0.f;
+        }
+        for (int e = tid; e < kRtOut * kRtK; e += 256) {
+          // consecutive threads take consecutive elements of the weight's rows
+          const int f = kDx ? e / kRtK : e % kRtOut, cc = kDx ? e % kRtK : e / kRtOut;
+          float v = 0.f;
+          if (f < no && cc < nc)
+            v = kDx ? ld_elem(W + ((long long)g * G + o_lo + f) * ldw + (long long)m * L + c0 + cc)
+                    : ld_elem(W + ((long long)m * L + c0 + cc) * ldw + (long long)g * G + o_lo + f);
+          bs[f][cc] = v;
+        }
+        __syncthreads();
+        // a thread whose first slot is past the kept rows has none (slots ty + 16 u)
+        for (int cc = 0; cc < (ty < n ? nc : 0); ++cc) {
+          float av[4], bv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            av[u] = as[ty + 16 * u][cc];
+            bv[u] = bs[tx + 16 * u][cc];
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) part[u][v] = fmaf(av[u], bv[v], part[u][v]);
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int sl = ty + 16 * u;
+        if (sl < n) {
+          const int i = s_idx[sl];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc_s[i][tx + 16 * v] += part[u][v];
+        }
+      }
+    }
+    __syncthreads();  // before the masks and the packed rows are rewritten
+  }
+  for (int e = tid; e < kRtRows * kRtOut; e += 256) {
+    const int i = e / kRtOut, f = e - i * kRtOut;
+    if (i < nr && f < no && s_t[i] >= 0) {
+      T* out = O + (r0 + i) * ldo + (long long)g * G + o_lo + f;
+      float v = acc_s[i][f];
+      if (accumulate) v += ld_elem(out);
+      st_elem(out, v);
+    }
+  }
+}
+
+// Launches k_rows_tiled when the rows fill at least half a tile, q is small
+// enough and the grid fits; returns false (nothing launched) otherwise.  Each
+// of the q contraction groups stages its whole weight slice whatever the
+// number of rows it applies to, so the tiles pay off for small q only: the
+// projection at q <= 8 (Q2xQ2 pilot shape 4.06 -> 1.25 ms; at q = 16 one
+// output a thread was faster), dX at q <= 32 (q = 16: 1.51 -> 0.30 ms).
+template <bool kDx>
+static bool launch_rows_tiled(int law, int q, const RowTypes& rt, long long row_begin, long long rows,
+                              const aal_mat& A, const aal_mat& W, const aal_mat& O, int L, int G,
+                              int accumulate, cudaStream_t s) {
+  const long long n = rows - row_begin;
+  const long long gx = (long long)q * ((G + kRtOut - 1) / kRtOut), gy = (n + kRtRows - 1) / kRtRows;
+  if (q > (kDx ? 32 : 8)) return false;
+  if (n < kRtRows / 2 || G <= 0 || gx > 0x7fffffffLL || gy > 65535) return false;
+  const dim3 grd((unsigned)gx, (unsigned)gy);
+  if (A.dtype == AAL_F32)
+    k_rows_tiled<float, kDx><<<grd, 256, 0, s>>>(law, q, rt, row_begin, rows, (const float*)A.ptr, A.ld,
+                                                 (const float*)W.ptr, W.ld, (float*)O.ptr, O.ld, L, G,
+                                                 accumulate);
+  else
+    k_rows_tiled<__nv_bfloat16, kDx><<<grd, 256, 0, s>>>(
+        law, q, rt, row_begin, rows, (const __nv_bfloat16*)A.ptr, A.ld, (const __nv_bfloat16*)W.ptr, W.ld,
+        (__nv_bfloat16*)O.ptr, O.ld, L, G, accumulate);
+  return true;
+}
+
+// The same dW on tiles that each lie inside one block (a, k): up to 64 of
+// group a's features by up to 64 of group k's columns, 256 threads of 4 x 4
+// outputs.  The tile walks the rows 32 at a time; a warp keeps the rows of the
+// step whose type t has a in S(t, k), packed to the front of shared memory
+// with their X and dY slices, so the tile does only the products the table
+// asks for (every row for a diagonal block, under Q_q the rows of type a or k
+// for the others) with every operand read once per tile.
+constexpr int kDwTile = 64, kDwRows = 32;
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_dw_tiled(int law, int q, RowTypes rt, long long rows,
+                                                      const T* __restrict__ X, long long ldx,
+                                                      const T* __restrict__ dY, long long ldy,
+                                                      T* __restrict__ dW, long long ldw, int bi, int bo,
+                                                      int accumulate) {
+  __shared__ float xs[kDwRows][kDwTile];
+  __shared__ float ys[kDwRows][kDwTile];
+  __shared__ long long rs[kDwRows];
+  __shared__ int s_n;
+  const int jt_per = (bi + kDwTile - 1) / kDwTile, ct_per = (bo + kDwTile - 1) / kDwTile;
+  const int a = (int)(blockIdx.x / jt_per), k = (int)(blockIdx.y / ct_per);
+  const int j_lo = (int)(blockIdx.x - (unsigned)a * jt_per) * kDwTile;  // within group a
+  const int c_lo = (int)(blockIdx.y - (unsigned)k * ct_per) * kDwTile;  // within group k
+  const int nj = bi - j_lo < kDwTile ? bi - j_lo : kDwTile;
+  const int nc = bo - c_lo < kDwTile ? bo - c_lo : kDwTile;
+  const long long j0 = (long long)a * bi + j_lo, c0 = (long long)k * bo + c_lo;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  float acc[4][4] = {};
+  for (long long r0 = 0; r0 < rows; r0 += kDwRows) {
+    if (tid < 32) {
+      const long long r = r0 + tid;
+      const int t = r < rows ? row_type(rt, r) : -1;
+      const bool keep = t >= 0 && in_table(law, t, k, a);
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) rs[__popc(m & ((1u << tid) - 1u))] = r;
+      if (tid == 0) s_n = __popc(m);
+    }
+    __syncthreads();
+    const int n = s_n;
+    for (int e = tid; e < n * kDwTile; e += 256) {
+      const int i = e / kDwTile, x = e - i * kDwTile;
+      const long long r = rs[i];
+      xs[i][x] = x < nj ? ld_elem(X + r * ldx + j0 + x) : 0.f;
+      ys[i][x] = x < nc ? ld_elem(dY + r * ldy + c0 + x) : 0.f;
+    }
+    __syncthreads();
+    for (int i = 0; i < n; ++i) {
+      float xv[4], yv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        xv[u] = xs[i][ty + 16 * u];
+        yv[u] = ys[i][tx + 16 * u];
+      }
+#pragma unroll
+      for (int uj = 0; uj < 4; ++uj)
+#pragma unroll
+        for (int uc = 0; uc < 4; ++uc) acc[uj][uc] = fmaf(xv[uj], yv[uc], acc[uj][uc]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int uj = 0; uj < 4; ++uj) {
+    const int jj = ty + 16 * uj;
+    if (jj >= nj) continue;
+#pragma unroll
+    for (int uc = 0; uc < 4; ++uc) {
+      const int cc = tx + 16 * uc;
+      if (cc >= nc) continue;
+      T* out = dW + (j0 + jj) * ldw + c0 + cc;
+      float v = acc[uj][uc];
+      if (accumulate) v += ld_elem(out);
+      st_elem(out, v);
+    }
+  }
+}
+
 // Z[row, col] = sum_{a in S(i, k)} sum_j X[row, a*b + j] W[a*b + j, col],
 // i = row / b, k = col / b.
 template <typename T>
@@ -173,6 +384,11 @@ aal_status simt_project_rows(int law, int q, const RowTypes& rt, long long row_b
   const long long rows = X.rows, dout = W.cols;
   const int bi = (int)(X.cols / q), bo = (int)(dout / q);
   if (rows <= row_begin || dout == 0) return AAL_OK;
+  if (launch_rows_tiled<false>(law, q, rt, row_begin, rows, X, W, Y, bi, bo, 0, s)) {
+    note_launch();
+    return cuda_status(cudaGetLastError());
+  }
+  // a few rows (decode) or a grid too large for the tiles: one thread per output
   dim3 blk(32, 8);
   if (!grid_ok(dout, rows - row_begin, blk)) return AAL_ERR_UNSUPPORTED;
   dim3 grd = grid2(dout, rows - row_begin, blk);
@@ -219,6 +435,10 @@ aal_status simt_project_bwd_dx(int law, int q, const RowTypes& rt, const aal_mat
   const long long rows = dY.rows, din = W.rows;
   const int bi = (int)(din / q), bo = (int)(W.cols / q);
   if (rows == 0 || din == 0) return AAL_OK;
+  if (launch_rows_tiled<true>(law, q, rt, 0, rows, dY, W, dX, bo, bi, accumulate, s)) {
+    note_launch();
+    return cuda_status(cudaGetLastError());
+  }
   dim3 blk(32, 8);
   if (!grid_ok(din, rows, blk)) return AAL_ERR_UNSUPPORTED;
   dim3 grd = grid2(din, rows, blk);
@@ -259,6 +479,22 @@ aal_status simt_project_bwd_dw(int law, int q, const RowTypes& rt, const aal_mat
   const long long rows = X.rows, din = dW.rows, dout = dW.cols;
   const int bi = (int)(din / q), bo = (int)(dout / q);
   if (din == 0 || dout == 0) return AAL_OK;
+  const long long gx = (long long)q * ((bi + kDwTile - 1) / kDwTile);
+  const long long gy = (long long)q * ((bo + kDwTile - 1) / kDwTile);
+  if (gx <= 0x7fffffffLL && gy <= 65535) {
+    const dim3 grd((unsigned)gx, (unsigned)gy);
+    if (X.dtype == AAL_F32)
+      k_bwd_dw_tiled<float><<<grd, 256, 0, s>>>(law, q, rt, rows, (const float*)X.ptr, X.ld,
+                                                (const float*)dY.ptr, dY.ld, (float*)dW.ptr, dW.ld, bi,
+                                                bo, accumulate);
+    else
+      k_bwd_dw_tiled<__nv_bfloat16><<<grd, 256, 0, s>>>(
+          law, q, rt, rows, (const __nv_bfloat16*)X.ptr, X.ld, (const __nv_bfloat16*)dY.ptr, dY.ld,
+          (__nv_bfloat16*)dW.ptr, dW.ld, bi, bo, accumulate);
+    note_launch();
+    return cuda_status(cudaGetLastError());
+  }
+  // more tile columns than a grid's y extent holds: one thread per output
   dim3 blk(32, 8);
   if (!grid_ok(dout, din, blk)) return AAL_ERR_UNSUPPORTED;
   dim3 grd = grid2(dout, din, blk);

@@ -492,6 +492,36 @@ def test_swiglu_bwd_split_heavy_tiles():
     assert got == TENSOR
 
 
+# The general path's dW runs on tiles inside one block (a, k): groups that are
+# not multiples of the 64-wide tile, steps of 32 rows with a short last one,
+# both laws, accumulation, q = 1.
+@pytest.mark.parametrize("law,q,M,din,dout,explicit,accumulate", [
+    ("Q", 3, 301, 300, 210, True, False),      # 100 x 70 blocks: partial tiles
+    ("Q", 8, 1000, 512, 64, False, True),      # 64 x 8 blocks, dW accumulated
+    ("Q2xQ2", 4, 77, 320, 80, True, False),    # 80 x 20 blocks
+    ("Q", 1, 45, 96, 48, False, False),        # one group: dense
+])
+def test_general_path_backward_tiles(law, q, M, din, dout, explicit, accumulate):
+    edx, edw, path = run_bwd(law, q, M, din, dout, "f32", explicit=explicit, accumulate=accumulate,
+                             seed=M, policy=GENERAL)
+    assert edx <= TOL["f32"] and edw <= TOL["f32"] and path == GENERAL, (edx, edw, path)
+
+
+# The general path's projection and dX run on 64-row tiles that keep, for each
+# group of the contraction, only the rows the table applies it to: a partial
+# last row tile, groups narrower or wider than a tile, both laws.
+@pytest.mark.parametrize("law,q,M,din,dout,explicit,seq_len", [
+    ("Q", 3, 301, 300, 210, True, None),
+    ("Q2xQ2", 4, 77, 320, 80, True, None),
+    ("Q", 8, 1000, 512, 64, False, 37),
+    ("Q", 5, 130, 80, 650, False, 130),
+])
+def test_general_path_projection_tiles(law, q, M, din, dout, explicit, seq_len):
+    err, path = run_project(law, q, M, din, dout, "f32", seq_len=seq_len, explicit=explicit, seed=M,
+                            policy=GENERAL)
+    assert err <= TOL["f32"] and path == GENERAL, (err, path)
+
+
 def test_general_path_matches_oracle():
     err, path = run_project("Q", 16, 2048, 2048, 768, "bf16", seq_len=2048, policy=GENERAL)
     assert err <= TOL["bf16"] and path == aal.AAL_PATH_GENERAL
