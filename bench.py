@@ -727,6 +727,9 @@ class ExplicitTypes:
             s["H"] = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
             s["Y"] = torch.empty(M, D, dtype=torch.bfloat16, device="cuda")
             s["ws"] = torch.empty(n, dtype=torch.uint8, device="cuda")
+            if self.swiglu:  # the dense comparison's pre-activations
+                s["G"] = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+                s["U"] = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
             self.sets.append(s)
 
     def kernel_model(self, name):
@@ -760,10 +763,15 @@ class ExplicitTypes:
         aal.aal_set_workspace(None)
 
     def dense_step(self, i):
+        """The same products dense: H = X Wg (projections), or G = X Wg,
+        U = X Wu, H = silu(G) * U (SwiGLU); then Y = H Wd."""
         s = self.sets[i % len(self.sets)]
-        torch.matmul(s["X"], s["Wg"], out=s["H"])
         if self.swiglu:
-            torch.matmul(s["X"], s["Wu"], out=s["H"])
+            torch.matmul(s["X"], s["Wg"], out=s["G"])
+            torch.matmul(s["X"], s["Wu"], out=s["U"])
+            torch.mul(torch.nn.functional.silu(s["G"], inplace=True), s["U"], out=s["H"])
+        else:
+            torch.matmul(s["X"], s["Wg"], out=s["H"])
         torch.matmul(s["H"], s["Wd"], out=s["Y"])
 
     def oracle_sample(self, rows):
