@@ -280,3 +280,17 @@ def test_backward_workspace_sizes():
                                   2048, 768) == 0
     with pytest.raises(ValueError):
         aal.aal_workspace_size(5, "Q", 16, rule, 2048, 2048, 768)
+
+
+def test_every_environment_switch_is_documented():
+    # each AAL_* variable the library reads appears in the header's list of switches
+    import glob
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    read = set()
+    for f in glob.glob(os.path.join(root, "associative_algebra_block_b200", "csrc", "*.cu")):
+        read |= set(re.findall(r'getenv\("(AAL_[A-Z0-9_]+)"\)', open(f).read()))
+    header = open(os.path.join(root, "include", "aal.h")).read()
+    documented = set(re.findall(r"(AAL_[A-Z0-9_]+)=", header))
+    assert read, "no switches found"
+    assert read <= documented, sorted(read - documented)
