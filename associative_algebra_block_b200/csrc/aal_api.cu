@@ -114,6 +114,9 @@ static cudaStream_t fork_side(cudaStream_t s) {
   for (SideStream& e : t_side)
     if (e.dev == dev) { ss = &e; break; }
   if (!ss) {
+    // created outside a capture only (a failing call inside one would end it)
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
     for (SideStream& e : t_side)
       if (e.dev < 0) { ss = &e; break; }
     if (!ss) return nullptr;

@@ -286,8 +286,9 @@ AAL_API aal_status aal_square_product(int32_t law, int32_t q, aal_mat X, aal_mat
  * is forked from and joined back to the call's stream by event records and
  * stream waits (so the call also captures into a CUDA graph), and the call's
  * stream orders everything as before.  The second stream and its two events
- * are created by a thread's first such call on a device (outside a capture,
- * ideally) and kept for the thread's lifetime.  The second stream's partial sums sit
+ * are created by a thread's first such call on a device outside a graph
+ * capture and kept for the thread's lifetime; a call captured before that
+ * keeps every launch on the call's stream.  The second stream's partial sums sit
  * after the first stream's in the workspace, and aal_workspace_size covers
  * that layout.
  *
